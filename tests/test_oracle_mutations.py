@@ -1,0 +1,61 @@
+"""Plant plausible mistakes in a copy of the oracle and check the pins fail.
+
+Each mutation edits one expression of ``oracle/oracle.c`` (a sign, a bit
+order, an index, a dropped term), compiles the edited copy into a temporary
+library, and runs ``tests/test_oracle.py`` against it in a subprocess.  The
+pins must reject every mutant.  The real oracle is never modified.
+"""
+
+import os
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+MUTATIONS = [
+    ("sign convention", "? +1 : -1;", "? -1 : +1;"),
+    ("bit order within a byte", "(row_bits[j >> 3] >> (j & 7))", "(row_bits[j >> 3] >> (7 - (j & 7)))"),
+    ("salient term dropped", "Wrow[w->s_idx[t]] += ar * ac * sign_at(bits, t);",
+     "Wrow[w->s_idx[t]] += 0.0 * ar * ac * sign_at(bits, t);"),
+    ("salient column index", "Wrow[w->s_idx[t]] += ar", "Wrow[t] += ar"),
+    ("alpha_c indexed backwards", "w->alpha_c[(size_t)k * N + j] : 1.0;\n            Wrow",
+     "w->alpha_c[(size_t)k * N + (N - 1 - j)] : 1.0;\n            Wrow"),
+    ("alpha_r of base 0 for every base", "const double ar = w->alpha_r[(size_t)k * M + i];\n        for (int64_t j",
+     "const double ar = w->alpha_r[i];\n        for (int64_t j"),
+    ("LUT entry sign", "s += ((p >> t) & 1) ? z : -z;", "s += ((p >> t) & 1) ? -z : z;"),
+    ("LUT pattern bit order", "p |= (int64_t)bit << t;", "p |= (int64_t)bit << (g - 1 - t);"),
+    ("LUT salient term dropped", "acc += w->s_alpha_r[(size_t)k * M + i] * s;", "acc += 0.0 * s;"),
+    ("fp16 exponent bias", "e - 25);", "e - 24);"),
+    ("last column dropped", "acc += Wrow[j] * xb[j];", "if (j + 1 < N) acc += Wrow[j] * xb[j];"),
+    ("tolerance magnitude signed", "mag += fabs(Wrow[j] * xb[j]);", "mag += Wrow[j] * xb[j];"),
+    ("salient x gather", "x_S[t] = x[s_idx[t]];", "x_S[t] = x[t];"),
+]
+
+
+def _run_mutant(name, old, new, workdir):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for '{name}' not unique"
+    tag = "".join(c if c.isalnum() else "_" for c in name)
+    mutated = os.path.join(workdir, f"oracle_{tag}.c")
+    with open(mutated, "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(workdir, f"liboracle_{tag}.so")
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", lib,
+                    mutated, "-lm"], check=True)
+    env = dict(os.environ, FB_ORACLE_LIB=lib, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle.py"),
+                        "-x", "-q", "-p", "no:cacheprovider"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    return name, r.returncode, r.stdout[-1500:]
+
+
+def test_pins_reject_every_mutant(tmp_path):
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        results = list(ex.map(lambda m: _run_mutant(*m, str(tmp_path)), MUTATIONS))
+    accepted = [(n, out) for n, rc, out in results if rc == 0]
+    assert not accepted, "pins accepted mutants: " + "; ".join(n for n, _ in accepted)
+    assert len(results) == len(MUTATIONS)
