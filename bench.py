@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-1 LUT binary GEMV on B200.
+
+Workload (the headline): M = N = 4096, K = 2 global +/-1 bases, g = 4, 128
+salient columns with 2 extra bases, batch 1, fp16 x ~ N(0,1),
+alpha ~ |N(0,0.02)| + 1e-3.  64 distinct weight sets of that shape (285 MB,
+more than twice the 126 MB L2) are rotated so every GEMV streams its weights
+from HBM.  One step = 1024 back-to-back GEMVs (16 passes over the 64 sets),
+captured in a CUDA graph of fb_gemv launches with programmatic dependent
+launch; each GEMV may depend on the previous one's output (x is read only
+after the previous kernel completes).
+
+Printed: one JSON line (rank 0).  value = achieved GB/s of algorithmic bytes
+(packed planes, scales, salient data, x, y) over all ranks; also GEMV us, the
+g = 8 variant on the same weights, the 7B-shaped decode step (224 GEMVs), the
+roofline of the GEMV kernel against the measured HBM peak, e2e through the
+Python API with host buffers, and the fp64 CPU oracle as baseline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GEMV µs & achieved HBM GB/s (% peak) at 4096×4096 K=2; 7B-shaped step ms"
+WEIGHT_SETS = 64
+PASSES_PER_STEP = 16
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-7b", action="store_true", help="skip the 7B-shaped step measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for f in ("lut_binary_gemv_b200/csrc/gemv.cu", "lut_binary_gemv_b200/csrc/fb_internal.cuh"):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel_tag):
+    """DRAM bytes per launch from the committed ncu summary, only if it was
+    taken on the current kernel source."""
+    try:
+        d = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
+        e = d[kernel_tag]
+        if e["source_sha256"] == source_digest():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = os.path.join("/tmp", f"fb_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu_id)], stdout=open(self.out, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.out):
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+    if args.impl == "ours":
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def workload_config():
+    return {"workload": "layer_4096x4096_k2_g4_s128", "M": 4096, "N": 4096, "K": 2, "g": 4, "nS": 128,
+            "Ks": 2, "batch": 1, "x_dtype": "f16", "weight_sets": WEIGHT_SETS,
+            "gemvs_per_step": WEIGHT_SETS * PASSES_PER_STEP,
+            "l2": "inputs larger than L2: 64 distinct weight sets (285 MB) rotated, no flush",
+            "launch": "CUDA graph of fb_gemv, programmatic dependent launch, x read after the wait"}
+
+
+# --------------------------------------------------------------------------
+def cpu_baseline(seconds):
+    """The fp64 oracle (dense dequantisation + fp64 dot) on this host's cores."""
+    import oracle
+    import workloads as wl
+    p = wl.layer4096()
+    w = oracle.OracleWeights.from_problem(p)
+    x = oracle.x_to_f64(p.x, p.x_dtype)
+    oracle.gemv(w, x)                        # warm (page in, thread pool)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.gemv(w, x)
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+    per = dt / n
+    return {"value": round(p.algorithmic_bytes() / per / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{n} full 4096x4096 K=2 GEMVs (all rows) of the same workload, "
+            f"{per * 1e3:.1f} ms each", "ms_per_gemv": round(per * 1e3, 3)}
+
+
+def run_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return                              # the oracle runs once, on rank 0's host
+
+    import oracle
+    import workloads as wl
+    p = wl.layer4096()
+    w = oracle.OracleWeights.from_problem(p)
+    x = oracle.x_to_f64(p.x, p.x_dtype)
+    oracle.gemv(w, x)
+    t1 = time.perf_counter()
+    oracle.gemv(w, x)
+    one = time.perf_counter() - t1
+    # each step: a bounded row sample so the whole run stays within a few minutes
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rows = p.M if one <= budget else max(32, int(p.M * budget / one) // 32 * 32)
+    sel = np.arange(rows)
+    for _ in range(args.warmup):
+        oracle.gemv(w, x, sel)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gemv(w, x, sel)
+    dt = time.perf_counter() - t0
+    frac_rows = rows / p.M
+    gbs = p.algorithmic_bytes() * frac_rows * args.steps / dt / 1e9
+    cores = oracle.num_threads()
+    sample = f"rows 0..{rows - 1} of the 4096x4096 K=2 GEMV per step ({rows / p.M:.3f} of the matrix)"
+    line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(),
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+def make_sets(n, device):
+    import torch
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    Ws, xs, bytes_per = [], [], None
+    for r in range(n):
+        p = wl.layer4096(seed=1 if r == 0 else (1, r))
+        Ws.append(fb.Weights.from_problem(p, device=device))
+        xs.append(torch.from_numpy(p.x[0]).to(device))
+        bytes_per = p.algorithmic_bytes()
+    torch.cuda.synchronize()
+    return Ws, xs, bytes_per
+
+
+def capture(stream, body):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        body()                         # warm-up launch outside capture (sets kernel attributes)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            body()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(graph, stream, steps, warmup, world, sampler=None):
+    import torch
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    barrier(world)
+    ms = start.elapsed_time(end)
+    return max_over_ranks(ms, world), clocks
+
+
+def run_ours(args):
+    import torch
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    from lut_binary_gemv_b200 import build as fb_build
+
+    rank, world, local = dist_setup(args)
+    if rank == 0:
+        fb_build.build()
+    barrier(world)
+    device = f"cuda:{local}"
+    peak, peak_src = measured_peak()
+
+    Ws, xs, bytes_per = make_sets(WEIGHT_SETS, device)
+    ys = [torch.empty(4096, dtype=torch.float32, device=device) for _ in range(WEIGHT_SETS)]
+    ws = Ws[0].workspace()          # one workspace: launches are stream-ordered
+    stream = torch.cuda.Stream(device=device)
+
+    def step(g_override=None):
+        def body():
+            for _ in range(PASSES_PER_STEP):
+                for r in range(WEIGHT_SETS):
+                    W = Ws[r] if g_override is None else Wg[r]
+                    fb.fb_gemv(W, xs[r], y=ys[r], ws=ws, flags=fb.FB_GEMV_PDL)
+        return body
+
+    gemvs = WEIGHT_SETS * PASSES_PER_STEP
+    graph = capture(stream, step())
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_id = vis.split(",")[local] if vis else str(local)
+    sampler = ClockSampler(gpu_id)
+    ms, clocks = time_graph(graph, stream, args.steps, args.warmup, world, sampler)
+    us_per_gemv = ms * 1e3 / (args.steps * gemvs)
+    gbs_rank = bytes_per / (us_per_gemv * 1e-6) / 1e9
+    value = gbs_rank * world
+
+    # g = 8 tables on the same weights (the layout does not depend on g)
+    Wg = [W.with_g(8) for W in Ws]
+    graph8 = capture(stream, step(8))
+    ms8, _ = time_graph(graph8, stream, max(20, args.steps // 4), args.warmup, world)
+    us8 = ms8 * 1e3 / (max(20, args.steps // 4) * gemvs)
+    gbs8 = bytes_per / (us8 * 1e-6) / 1e9
+    del graph8
+
+    # e2e through the Python API: host x in, host y out, every step
+    n_e2e = WEIGHT_SETS
+    x_host = torch.stack([x.cpu() for x in xs]).pin_memory()
+    y_host = torch.empty((n_e2e, 4096), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x_host, device=device)
+    y_dev = torch.empty((n_e2e, 4096), dtype=torch.float32, device=device)
+    e2e_steps = max(10, args.steps // 10)
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            for r in range(n_e2e):
+                fb.fb_gemv(Ws[r], x_dev[r], y=y_dev[r], ws=ws)
+            y_host.copy_(y_dev, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        s1.synchronize()
+    ms_e2e = max_over_ranks(s0.elapsed_time(s1), world)
+    e2e_gbs = bytes_per * n_e2e * e2e_steps / (ms_e2e * 1e-3) / 1e9 * world
+
+    del graph
+    torch.cuda.synchronize()
+
+    step7b = None
+    if not args.no_7b:
+        step7b = bench_7b(args, device, stream, world, peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    traffic = ncu_traffic("gemv_g4_f16_layer4096")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(), parallelism=f"replicas{world}"),
+        "gemv_us": round(us_per_gemv, 4),
+        "roofline": {"bound": "hbm", "achieved": round(gbs_rank, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs_rank / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                     else "fallback 6.65 TB/s",
+                     "algorithmic_bytes_per_launch": bytes_per},
+        "variants": {"g8_pair_tables": {"gemv_us": round(us8, 4), "gbs": round(gbs8, 2),
+                                        "frac": round(gbs8 / peak, 4),
+                                        "note": "same weights, 256-entry tables over 8 columns"}},
+        "step_7b": step7b,
+        "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 4),
+                "note": f"{n_e2e} eager fb_gemv calls per step from Python, pinned host x in and y out"},
+        "gpu_launches": args.steps * gemvs,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def bench_7b(args, device, stream, world, peak):
+    """The 7B-shaped decode step: 32 layers x (q,k,v,o 4096x4096; gate, up
+    11008x4096; down 4096x11008), K=2, g=4, 3% salient, fresh fp16 x per GEMV;
+    224 GEMVs in one CUDA graph with programmatic dependent launch."""
+    import torch
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    Ws, xs, ys, total = [], [], [], 0
+    for layer in range(wl.STEP7B_LAYERS):
+        for m in range(len(wl.STEP7B_MATRICES)):
+            p = wl.step7b_matrix(layer, m)
+            Ws.append(fb.Weights.from_problem(p, device=device))
+            xs.append(torch.from_numpy(p.x[0]).to(device))
+            ys.append(torch.empty(p.M, dtype=torch.float32, device=device))
+            total += p.algorithmic_bytes()
+    nbytes = max(fb.fb_gemv_workspace_bytes(W) for W in Ws)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+    def body():
+        for W, x, y in zip(Ws, xs, ys):
+            fb.fb_gemv(W, x, y=y, ws=ws, flags=fb.FB_GEMV_PDL)
+
+    graph = capture(stream, body)
+    steps = max(30, args.steps // 4)
+    ms, _ = time_graph(graph, stream, steps, args.warmup, world)
+    per = ms / steps
+    gbs = total / (per * 1e-3) / 1e9
+    del graph
+    return {"ms": round(per, 5), "gbs": round(gbs, 2), "frac": round(gbs / peak, 4),
+            "algorithmic_bytes": total, "gemvs": len(Ws), "steps": steps}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/fluxbin.h declares, and rejects bad arguments with
+the documented status before touching the GPU."""
+
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import lut_binary_gemv_b200 as fb
+from lut_binary_gemv_b200 import build as fb_build
+from tests.layout_spec import pack_reference
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fluxbin.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA = range(6)
+
+
+@pytest.fixture(scope="module")
+def L():
+    fb_build.build()
+    return fb.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FB_API[^;{]*?\b(fb_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_five_hot_path_calls():
+    names = declared_functions()
+    for n in ("fb_pack", "fb_lut_build", "fb_vcm_gather", "fb_gemv", "fb_gemv_batched"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 12
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version(L):
+    for code, name in enumerate(["FB_OK", "FB_ERR_INVALID_VALUE", "FB_ERR_UNSUPPORTED",
+                                 "FB_ERR_MISALIGNED", "FB_ERR_WORKSPACE", "FB_ERR_CUDA"]):
+        assert fb.fb_status_string(code) == name
+    assert L.fb_abi_version() == 1
+
+
+def test_packed_words(L):
+    assert fb.fb_packed_words(2, 4096, 4096) == 2 * 4096 * 4096 // 32
+    assert fb.fb_packed_words(3, 33, 800) == 3 * 64 * 800 // 32
+    assert fb.fb_packed_words(1, 1, 32) == 32
+    for bad in [(0, 8, 32), (5, 8, 32), (1, 0, 32), (1, 8, 48), (1, 8, 0), (1, 8, 16)]:
+        assert fb.fb_packed_words(*bad) == 0
+
+
+FAKE = 0x10000   # an aligned non-null address; host-only calls never dereference it
+
+
+def fake_weights(M=256, N=512, K=2, g=4, nS=0, Ks=2, **over):
+    s = fb.FbWeightsStruct(M=M, N=N, K=K, g=g, planes=FAKE, alpha_r=FAKE, alpha_c=FAKE, nS=nS,
+                           Ks=Ks if nS else 0, s_idx=FAKE if nS else None,
+                           s_planes=FAKE if nS else None, s_alpha_r=FAKE if nS else None,
+                           s_alpha_c=FAKE if nS else None)
+    for k, v in over.items():
+        setattr(s, k, v)
+    return s
+
+
+def ws_bytes(L, s, batch=1):
+    return L.fb_gemv_workspace_bytes(C.byref(s), batch)
+
+
+def test_workspace_bytes_formula(L):
+    # partials: batch * panels(per base) * M_pad floats; counters: batch * chunks
+    s = fake_weights(M=4096, N=4096, K=2, nS=128, Ks=2)
+    V = 16 * 2 + 1 * 2
+    assert ws_bytes(L, s) == V * 4096 * 4 + 128 * 4
+    s = fake_weights(M=100, N=800, K=3)
+    V, M_pad = 4 * 3, 128
+    part = V * M_pad * 4
+    assert ws_bytes(L, s, 4) == (4 * part + 255) // 256 * 256 + 256
+    assert ws_bytes(L, s, 0) == 0 and ws_bytes(L, s, 65) == 0
+    assert ws_bytes(L, fake_weights(g=3)) == 0
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(g=3), INVALID), (dict(g=16), INVALID), (dict(N=48), INVALID), (dict(K=0), INVALID),
+    (dict(K=5), INVALID), (dict(M=0), INVALID), (dict(planes=None), INVALID),
+    (dict(alpha_r=None), INVALID), (dict(planes=FAKE + 4), MISALIGNED),
+    (dict(alpha_r=FAKE + 2), MISALIGNED), (dict(alpha_c=FAKE + 1), MISALIGNED),
+    (dict(nS=600), INVALID), (dict(nS=-1), INVALID),
+])
+def test_gemv_rejects_bad_weights(L, over, status):
+    s = fake_weights(**over)
+    y = FAKE
+    assert L.fb_gemv(C.byref(s), FAKE, 1, y, FAKE, 1 << 30, 0, None) == status
+
+
+def test_gemv_rejects_bad_salient(L):
+    s = fake_weights(nS=10, Ks=0)
+    assert L.fb_gemv(C.byref(s), FAKE, 1, FAKE, FAKE, 1 << 30, 0, None) == INVALID
+    s = fake_weights(nS=10, Ks=5)
+    assert L.fb_gemv(C.byref(s), FAKE, 1, FAKE, FAKE, 1 << 30, 0, None) == INVALID
+    s = fake_weights(nS=10, Ks=2)
+    s.s_idx = None
+    assert L.fb_gemv(C.byref(s), FAKE, 1, FAKE, FAKE, 1 << 30, 0, None) == INVALID
+    s = fake_weights(nS=10, Ks=2)
+    s.s_planes = FAKE + 8
+    assert L.fb_gemv(C.byref(s), FAKE, 1, FAKE, FAKE, 1 << 30, 0, None) == MISALIGNED
+
+
+def test_gemv_rejects_bad_call_arguments(L):
+    s = fake_weights()
+    need = ws_bytes(L, s)
+    W = C.byref(s)
+    assert L.fb_gemv(None, FAKE, 1, FAKE, FAKE, need, 0, None) == INVALID
+    assert L.fb_gemv(W, None, 1, FAKE, FAKE, need, 0, None) == INVALID
+    assert L.fb_gemv(W, FAKE, 1, None, FAKE, need, 0, None) == INVALID
+    assert L.fb_gemv(W, FAKE, 7, FAKE, FAKE, need, 0, None) == INVALID      # dtype
+    assert L.fb_gemv(W, FAKE, 1, FAKE, FAKE, need, 4, None) == INVALID      # unknown flag
+    assert L.fb_gemv(W, FAKE + 1, 1, FAKE, FAKE, need, 0, None) == MISALIGNED
+    assert L.fb_gemv(W, FAKE, 0, FAKE + 2, FAKE, need, 0, None) == MISALIGNED
+    assert L.fb_gemv(W, FAKE, 1, FAKE, None, need, 0, None) == WORKSPACE
+    assert L.fb_gemv(W, FAKE, 1, FAKE, FAKE, need - 1, 0, None) == WORKSPACE
+    assert L.fb_gemv(W, FAKE, 1, FAKE, FAKE + 8, need, 0, None) == WORKSPACE
+    b = L.fb_gemv_batched
+    assert b(W, FAKE, 1, 0, 512, FAKE, 256, FAKE, need, 0, None) == INVALID   # batch 0
+    assert b(W, FAKE, 1, 65, 512, FAKE, 256, FAKE, 1 << 30, 0, None) == INVALID
+    assert b(W, FAKE, 1, 2, 500, FAKE, 256, FAKE, 1 << 30, 0, None) == INVALID  # ldx < N
+    assert b(W, FAKE, 1, 2, 512, FAKE, 200, FAKE, 1 << 30, 0, None) == INVALID  # ldy < M
+    assert b(W, FAKE, 1, 2, 512, FAKE, 256, FAKE, ws_bytes(L, s, 2) - 4, 0, None) == WORKSPACE
+
+
+def test_other_entry_points_reject_bad_arguments(L):
+    assert L.fb_pack(None, 1, 8, 32, FAKE, None) == INVALID
+    assert L.fb_pack(FAKE, 1, 8, 40, FAKE, None) == INVALID
+    assert L.fb_pack(FAKE, 1, 8, 32, FAKE + 4, None) == MISALIGNED
+    assert L.fb_pack(FAKE + 1, 1, 8, 32, FAKE, None) == MISALIGNED
+    assert L.fb_pack_bits(FAKE, 5, 8, 32, FAKE, None) == INVALID
+    assert L.fb_unpack(FAKE, 1, 8, 32, None, None) == INVALID
+    assert L.fb_lut_build(FAKE, 1, None, 2, 64, 3, FAKE, None) == INVALID
+    assert L.fb_lut_build(FAKE, 9, None, 2, 64, 4, FAKE, None) == INVALID
+    assert L.fb_lut_build(FAKE + 1, 1, None, 2, 64, 4, FAKE, None) == MISALIGNED
+    assert L.fb_vcm_gather(FAKE, 1, 1, 64, 64, FAKE, 10, 8, FAKE, 32, None) == INVALID   # nS_pad < nS
+    assert L.fb_vcm_gather(FAKE, 1, 1, 64, 32, FAKE, 10, 32, FAKE, 32, None) == INVALID  # ld_src < n_src
+    assert L.fb_vcm_gather(FAKE, 1, 1, 64, 64, None, 10, 32, FAKE, 32, None) == INVALID
+    assert L.fb_validate_weights(C.byref(fake_weights(g=5))) == INVALID
+    assert L.fb_validate_weights(None) == INVALID
+
+
+def test_layout_spec_is_a_bijection():
+    """Every (base, row, column) lands on its own bit of the packed buffer."""
+    rng = np.random.default_rng(0)
+    for K, M, N in [(1, 32, 32), (2, 40, 288), (1, 64, 800), (3, 7, 416)]:
+        n = K * ((M + 31) // 32 * 32) * N // 8
+        seen = np.zeros(n * 8, dtype=np.int64)
+        for k in range(K):
+            for r in rng.choice(M, min(M, 5), replace=False):
+                for c in range(N):
+                    s = -np.ones((K, M, N), np.int8)
+                    s[k, r, c] = 1
+                    bits = np.unpackbits(pack_reference(s), bitorder="little")
+                    pos = np.flatnonzero(bits)
+                    assert len(pos) == 1
+                    seen[pos[0]] += 1
+        assert seen.max() == 1
