@@ -7,8 +7,11 @@ alpha ~ |N(0,0.02)| + 1e-3.  64 distinct weight sets of that shape (285 MB,
 more than twice the 126 MB L2) are rotated so every GEMV streams its weights
 from HBM.  One step = 1024 back-to-back GEMVs (16 passes over the 64 sets),
 captured in a CUDA graph of fb_gemv launches with programmatic dependent
-launch; each GEMV may depend on the previous one's output (x is read only
-after the previous kernel completes).
+launch.  Every GEMV has its own freshly drawn x and its own y, so the GEMVs
+are independent and are launched with FB_GEMV_INDEPENDENT (each may overlap
+its predecessor; completion order is kept).  The same graph with every GEMV
+waiting for its predecessor before reading x (a dependent decode chain) is
+timed too and reported as "dependent_chain".
 
 Printed: one JSON line (rank 0).  value = achieved GB/s of algorithmic bytes
 (packed planes, scales, salient data, x, y) over all ranks; also GEMV us, the
@@ -49,6 +52,8 @@ def parse():
     ap.add_argument("--no-7b", action="store_true", help="skip the 7B-shaped step measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="small case for ncu: 32 weight sets (142 MB), one pass per step, headline graph only")
     return ap.parse_args()
 
 
@@ -170,7 +175,7 @@ def workload_config():
             "Ks": 2, "batch": 1, "x_dtype": "f16", "weight_sets": WEIGHT_SETS,
             "gemvs_per_step": WEIGHT_SETS * PASSES_PER_STEP,
             "l2": "inputs larger than L2: 64 distinct weight sets (285 MB) rotated, no flush",
-            "launch": "CUDA graph of fb_gemv, programmatic dependent launch, x read after the wait"}
+            "launch": "CUDA graph of fb_gemv, PDL + FB_GEMV_INDEPENDENT (fresh x and own y per GEMV)"}
 
 
 # --------------------------------------------------------------------------
@@ -295,21 +300,24 @@ def run_ours(args):
     device = f"cuda:{local}"
     peak, peak_src = measured_peak()
 
+    global WEIGHT_SETS, PASSES_PER_STEP
+    if args.profile:
+        WEIGHT_SETS, PASSES_PER_STEP = 32, 1
     Ws, xs, bytes_per = make_sets(WEIGHT_SETS, device)
     ys = [torch.empty(4096, dtype=torch.float32, device=device) for _ in range(WEIGHT_SETS)]
-    ws = Ws[0].workspace()          # one workspace: launches are stream-ordered
     stream = torch.cuda.Stream(device=device)
 
-    def step(g_override=None):
+    indep = fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT
+
+    def step(sets, flags):
         def body():
             for _ in range(PASSES_PER_STEP):
                 for r in range(WEIGHT_SETS):
-                    W = Ws[r] if g_override is None else Wg[r]
-                    fb.fb_gemv(W, xs[r], y=ys[r], ws=ws, flags=fb.FB_GEMV_PDL)
+                    fb.fb_gemv(sets[r], xs[r], y=ys[r], flags=flags)
         return body
 
     gemvs = WEIGHT_SETS * PASSES_PER_STEP
-    graph = capture(stream, step())
+    graph = capture(stream, step(Ws, indep))
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_id = vis.split(",")[local] if vis else str(local)
     sampler = ClockSampler(gpu_id)
@@ -317,14 +325,30 @@ def run_ours(args):
     us_per_gemv = ms * 1e3 / (args.steps * gemvs)
     gbs_rank = bytes_per / (us_per_gemv * 1e-6) / 1e9
     value = gbs_rank * world
+    del graph
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "gemv_us": round(us_per_gemv, 4),
+                              "gemvs": args.steps * gemvs}), flush=True)
+        return
 
+    def side(sets, flags):
+        g = capture(stream, step(sets, flags))
+        n = max(20, args.steps // 4)
+        t, _ = time_graph(g, stream, n, args.warmup, world)
+        us = t * 1e3 / (n * gemvs)
+        gbs = bytes_per / (us * 1e-6) / 1e9
+        return {"gemv_us": round(us, 4), "gbs": round(gbs, 2), "frac": round(gbs / peak, 4)}
+
+    # the same GEMVs as a dependent chain (each waits for the previous before reading x)
+    dependent = side(Ws, fb.FB_GEMV_PDL)
+    dependent["note"] = "each GEMV reads x only after the previous kernel completes"
     # g = 8 tables on the same weights (the layout does not depend on g)
     Wg = [W.with_g(8) for W in Ws]
-    graph8 = capture(stream, step(8))
-    ms8, _ = time_graph(graph8, stream, max(20, args.steps // 4), args.warmup, world)
-    us8 = ms8 * 1e3 / (max(20, args.steps // 4) * gemvs)
-    gbs8 = bytes_per / (us8 * 1e-6) / 1e9
-    del graph8
+    g8 = side(Wg, indep)
+    g8["note"] = "same weights, 256-entry tables over 8 columns"
+    g8_dep = side(Wg, fb.FB_GEMV_PDL)
+    g8["dependent_chain_gemv_us"] = g8_dep["gemv_us"]
 
     # e2e through the Python API: host x in, host y out, every step
     n_e2e = WEIGHT_SETS
@@ -337,7 +361,7 @@ def run_ours(args):
         def e2e_step():
             x_dev.copy_(x_host, non_blocking=True)
             for r in range(n_e2e):
-                fb.fb_gemv(Ws[r], x_dev[r], y=y_dev[r], ws=ws)
+                fb.fb_gemv(Ws[r], x_dev[r], y=y_dev[r])
             y_host.copy_(y_dev, non_blocking=True)
         for _ in range(3):
             e2e_step()
@@ -351,8 +375,6 @@ def run_ours(args):
         s1.synchronize()
     ms_e2e = max_over_ranks(s0.elapsed_time(s1), world)
     e2e_gbs = bytes_per * n_e2e * e2e_steps / (ms_e2e * 1e-3) / 1e9 * world
-
-    del graph
     torch.cuda.synchronize()
 
     step7b = None
@@ -375,9 +397,8 @@ def run_ours(args):
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                      else "fallback 6.65 TB/s",
                      "algorithmic_bytes_per_launch": bytes_per},
-        "variants": {"g8_pair_tables": {"gemv_us": round(us8, 4), "gbs": round(gbs8, 2),
-                                        "frac": round(gbs8 / peak, 4),
-                                        "note": "same weights, 256-entry tables over 8 columns"}},
+        "dependent_chain": dependent,
+        "variants": {"g8_pair_tables": g8},
         "step_7b": step7b,
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 4),
@@ -408,21 +429,23 @@ def bench_7b(args, device, stream, world, peak):
             xs.append(torch.from_numpy(p.x[0]).to(device))
             ys.append(torch.empty(p.M, dtype=torch.float32, device=device))
             total += p.algorithmic_bytes()
-    nbytes = max(fb.fb_gemv_workspace_bytes(W) for W in Ws)
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    def run(flags, steps):
+        def body():
+            for W, x, y in zip(Ws, xs, ys):
+                fb.fb_gemv(W, x, y=y, flags=flags)
+        graph = capture(stream, body)
+        ms, _ = time_graph(graph, stream, steps, args.warmup, world)
+        return ms / steps
 
-    def body():
-        for W, x, y in zip(Ws, xs, ys):
-            fb.fb_gemv(W, x, y=y, ws=ws, flags=fb.FB_GEMV_PDL)
-
-    graph = capture(stream, body)
     steps = max(30, args.steps // 4)
-    ms, _ = time_graph(graph, stream, steps, args.warmup, world)
-    per = ms / steps
+    per = run(fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT, steps)
+    per_dep = run(fb.FB_GEMV_PDL, steps)
     gbs = total / (per * 1e-3) / 1e9
-    del graph
     return {"ms": round(per, 5), "gbs": round(gbs, 2), "frac": round(gbs / peak, 4),
-            "algorithmic_bytes": total, "gemvs": len(Ws), "steps": steps}
+            "ms_dependent_chain": round(per_dep, 5),
+            "frac_dependent_chain": round(total / (per_dep * 1e-3) / 1e9 / peak, 4),
+            "algorithmic_bytes": total, "gemvs": len(Ws), "steps": steps,
+            "note": "224 GEMVs, fresh x per GEMV (independent); dependent chain: each waits for its predecessor"}
 
 
 def main():

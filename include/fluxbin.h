@@ -146,25 +146,30 @@ typedef struct fb_weights {
 FB_API fb_status fb_validate_weights(const fb_weights *W);
 
 /* fb_gemv_workspace_bytes: bytes of workspace fb_gemv / fb_gemv_batched need
- * for W at this batch size (0 if W is invalid).  Host only; independent of
- * the device.  The workspace holds per-panel fp32 partial sums and per
- * row-block arrival counters.  It must be zero-filled ONCE before its first
- * use (e.g. cudaMemset); every call leaves the counters at zero again.  Calls
- * that may overlap on the GPU must use different workspaces. */
+ * for W at this batch size.  The current kernels keep every partial sum in
+ * on-chip shared memory of a thread-block cluster, so this returns 0 and the
+ * ws / ws_bytes arguments may be NULL / 0 (they are kept for kernels that
+ * need scratch; a non-NULL ws is ignored).  Host only. */
 FB_API size_t fb_gemv_workspace_bytes(const fb_weights *W, int batch);
 
 /* Launch flags. */
-#define FB_GEMV_PDL 1u /* launch as a programmatic dependent launch: the kernel
-                          starts before the previous kernel in the stream ends
-                          and loads the weights (planes, scales, s_idx) early;
-                          it reads x, the workspace and y only after the
-                          previous kernel has completed.  Only valid when no
-                          kernel still running may write the weights. */
+#define FB_GEMV_PDL 1u /* programmatic dependent launch: the kernel may start
+                          before the previous kernel in the stream ends and
+                          loads its weights (planes, scales, s_idx) early; it
+                          reads x and writes y only after the previous kernel
+                          has completed.  Only valid when no kernel still
+                          running writes the weights. */
+#define FB_GEMV_INDEPENDENT 2u /* with FB_GEMV_PDL only: the previous kernel in
+                          the stream neither writes this call's x nor reads or
+                          writes its y, so the whole GEMV may overlap it; the
+                          kernel still completes only after the previous one,
+                          so ordering with later work is unchanged. */
 
 /* fb_gemv: y[i] = sum_j W_hat[i][j] * x[j] for i < M (batch 1), fp32 out,
  * overwriting y (beta = 0).  x: N elements of type t (2- or 4-byte aligned);
- * y: M floats, 4-byte aligned, must not alias x; ws: >= fb_gemv_workspace_bytes
- * (W, 1) bytes, 16-byte aligned (see above).  Table entries and all sums are
+ * y: M floats, 4-byte aligned, must not alias x; ws: see
+ * fb_gemv_workspace_bytes.  flags: 0 or FB_GEMV_PDL [| FB_GEMV_INDEPENDENT];
+ * anything else is FB_ERR_INVALID_VALUE.  Table entries and all sums are
  * fp32.  Deterministic: the same inputs give the same bits on every run. */
 FB_API fb_status fb_gemv(const fb_weights *W, const void *x, fb_dtype t, float *y, void *ws,
                   size_t ws_bytes, unsigned flags, void *stream);

@@ -21,7 +21,7 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "FbError", "Weights", "lib", "library_path", "FB_GEMV_PDL",
+    "FbError", "Weights", "lib", "library_path", "FB_GEMV_PDL", "FB_GEMV_INDEPENDENT",
     "fb_packed_words", "fb_pack", "fb_pack_bits", "fb_unpack", "fb_vcm_gather",
     "fb_lut_build", "fb_validate_weights", "fb_gemv_workspace_bytes", "fb_gemv",
     "fb_gemv_batched", "fb_status_string",
@@ -32,6 +32,7 @@ library_path = os.path.join(_HERE, "libfluxbin.so")
 
 FB_OK = 0
 FB_GEMV_PDL = 1
+FB_GEMV_INDEPENDENT = 2
 _DTYPES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 _STATUS = {0: "FB_OK", 1: "FB_ERR_INVALID_VALUE", 2: "FB_ERR_UNSUPPORTED", 3: "FB_ERR_MISALIGNED",
            4: "FB_ERR_WORKSPACE", 5: "FB_ERR_CUDA"}

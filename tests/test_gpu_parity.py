@@ -178,18 +178,43 @@ def test_gemv_deterministic_and_pdl():
     assert np.array_equal(a, b) and np.array_equal(a, c)
 
 
-def test_workspace_shared_by_different_weights():
+def test_interleaved_weights_and_flags():
+    """Different weight sets back to back, with every flag combination."""
     p1 = wl.make_problem(300, 1024, 2, nS=40, Ks=2, x_dtype="f16", seed=9)
     p2 = wl.make_problem(500, 512, 3, g=8, x_dtype="f32", seed=10)
     W1, W2 = fb.Weights.from_problem(p1), fb.Weights.from_problem(p2)
-    n = max(fb.fb_gemv_workspace_bytes(W1), fb.fb_gemv_workspace_bytes(W2))
-    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
-    for _ in range(3):
-        y1 = fb.fb_gemv(W1, x_tensor(p1)[0], ws=ws)
-        y2 = fb.fb_gemv(W2, x_tensor(p2)[0], ws=ws)
+    for flags in (0, fb.FB_GEMV_PDL, fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT):
+        for _ in range(3):
+            y1 = fb.fb_gemv(W1, x_tensor(p1)[0], flags=flags)
+            y2 = fb.fb_gemv(W2, x_tensor(p2)[0], flags=flags)
+        torch.cuda.synchronize()
+        check(p1, y1.cpu().numpy()[None].astype(np.float64))
+        check(p2, y2.cpu().numpy()[None].astype(np.float64))
+
+
+def test_independent_chain_in_graph_matches():
+    """Independent calls overlap each other; results must not change."""
+    ps = [wl.make_problem(700, 1280, 2, nS=33, Ks=2, x_dtype="f16", seed=20 + i) for i in range(6)]
+    Ws = [fb.Weights.from_problem(p) for p in ps]
+    xs = [x_tensor(p)[0] for p in ps]
+    ys = [torch.full((p.M,), float("nan"), device=DEV) for p in ps]
+    s = torch.cuda.Stream()
+    flags = fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT
+    with torch.cuda.stream(s):
+        for W, x, y in zip(Ws, xs, ys):
+            fb.fb_gemv(W, x, y=y, flags=flags)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(2):
+                for W, x, y in zip(Ws, xs, ys):
+                    fb.fb_gemv(W, x, y=y, flags=flags)
+    for y in ys:
+        y.fill_(float("nan"))
+    g.replay()
     torch.cuda.synchronize()
-    check(p1, y1.cpu().numpy()[None].astype(np.float64))
-    check(p2, y2.cpu().numpy()[None].astype(np.float64))
+    for p, y in zip(ps, ys):
+        check(p, y.cpu().numpy()[None].astype(np.float64))
 
 
 def test_gemv_in_cuda_graph():
@@ -197,7 +222,6 @@ def test_gemv_in_cuda_graph():
     W = fb.Weights.from_problem(p)
     x = x_tensor(p)[0]
     y = torch.empty(p.M, device=DEV)
-    W.workspace()
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         fb.fb_gemv(W, x, y=y, flags=fb.FB_GEMV_PDL)     # warm-up outside capture
