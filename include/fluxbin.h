@@ -125,7 +125,12 @@ FB_API fb_status fb_lut_build(const void *x, fb_dtype t, const float *alpha_c, i
 /* Weights of one M x N linear layer.  Host struct; every pointer in it is a
  * device pointer owned by the caller. */
 typedef struct fb_weights {
-    int M, N, K, g;              /* g: LUT group width used by fb_gemv */
+    int M, N, K, g;              /* g: LUT group width (1, 2, 4 or 8).  fb_gemv
+                                    looks up one weight byte (8 columns) per
+                                    table access for every g: each byte-table
+                                    entry is the sum of the byte's 8/g
+                                    g-column LUT entries, added pairwise, so g
+                                    fixes the grouping of the fp32 sums */
     const uint32_t *planes;      /* fb_pack(K, M, N) output, 16-byte aligned */
     const float *alpha_r;        /* [K][M] row scales */
     const float *alpha_c;        /* [K][N] column scales, or NULL for all ones */
@@ -170,7 +175,10 @@ FB_API size_t fb_gemv_workspace_bytes(const fb_weights *W, int batch);
  * y: M floats, 4-byte aligned, must not alias x; ws: see
  * fb_gemv_workspace_bytes.  flags: 0 or FB_GEMV_PDL [| FB_GEMV_INDEPENDENT];
  * anything else is FB_ERR_INVALID_VALUE.  Table entries and all sums are
- * fp32.  Deterministic: the same inputs give the same bits on every run. */
+ * fp32.  Deterministic: the same inputs give the same bits on every run.
+ * Weight copies are waited for with a bound (about 0.2 s); a kernel that
+ * gives up writes NaN into the rows it owns and raises bit 0 of
+ * fb_device_errors. */
 FB_API fb_status fb_gemv(const fb_weights *W, const void *x, fb_dtype t, float *y, void *ws,
                   size_t ws_bytes, unsigned flags, void *stream);
 
@@ -179,6 +187,25 @@ FB_API fb_status fb_gemv(const fb_weights *W, const void *x, fb_dtype t, float *
 FB_API fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtype t, int batch, int ldx,
                           float *Y, int ldy, void *ws, size_t ws_bytes, unsigned flags,
                           void *stream);
+
+/* fb_gemv_launch_plan: diagnostic, host only.  The launch shape fb_gemv /
+ * fb_gemv_batched use for W at this batch size and these flags (calls flagged
+ * FB_GEMV_INDEPENDENT get a throughput plan, others a latency plan) on a GPU
+ * with `sms` SMs:
+ * out[0] = CTAs per thread-block cluster, out[1] = chunks of 32 rows per row
+ * block, out[2] = row blocks, out[3] = warps per CTA, out[4] = dynamic shared
+ * memory bytes per CTA, out[5] = virtual panels (256-column panels x bases).
+ * out must hold 6 ints.  Returns FB_OK, or FB_ERR_INVALID_VALUE for invalid
+ * weights, batch, sms or flags. */
+FB_API fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned flags, int sms, int *out);
+
+/* fb_device_errors: synchronises the current device, then stores in *flags
+ * the error bits GEMV kernels have raised since the last clear (bit 0: a
+ * kernel gave up a bounded wait for one of its weight copies; the rows of
+ * that CTA were written as NaN), and clears them when clear != 0.  Returns
+ * FB_ERR_INVALID_VALUE for a null flags, FB_ERR_CUDA if the device reports an
+ * error, else FB_OK. */
+FB_API fb_status fb_device_errors(unsigned int *flags, int clear);
 
 /* Human-readable name of a status code (static string). */
 FB_API const char *fb_status_string(fb_status s);

@@ -24,7 +24,7 @@ __all__ = [
     "FbError", "Weights", "lib", "library_path", "FB_GEMV_PDL", "FB_GEMV_INDEPENDENT",
     "fb_packed_words", "fb_pack", "fb_pack_bits", "fb_unpack", "fb_vcm_gather",
     "fb_lut_build", "fb_validate_weights", "fb_gemv_workspace_bytes", "fb_gemv",
-    "fb_gemv_batched", "fb_status_string",
+    "fb_gemv_batched", "fb_status_string", "fb_gemv_launch_plan", "fb_device_errors",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -79,6 +79,8 @@ def lib() -> C.CDLL:
             "fb_gemv_workspace_bytes": (S, [W, I]),
             "fb_gemv": (I, [W, P, I, P, P, S, C.c_uint, P]),
             "fb_gemv_batched": (I, [W, P, I, I, I, P, I, P, S, C.c_uint, P]),
+            "fb_gemv_launch_plan": (I, [W, I, C.c_uint, I, P]),
+            "fb_device_errors": (I, [P, I]),
             "fb_status_string": (C.c_char_p, [I]),
             "fb_abi_version": (I, []),
         }
@@ -270,3 +272,20 @@ def fb_gemv_batched(W: Weights, X: torch.Tensor, Y: Optional[torch.Tensor] = Non
                                  Y.stride(0), ws.data_ptr(), ws.numel() * ws.element_size(), flags,
                                  _stream(X.device)), "fb_gemv_batched")
     return Y
+
+
+def fb_gemv_launch_plan(W, batch: int = 1, flags: int = 0, sms: int = 148) -> dict:
+    """The launch shape fb_gemv would use for W (a Weights or an
+    FbWeightsStruct: only its sizes and pointer alignment are read, so no GPU
+    is needed)."""
+    out = (C.c_int * 6)()
+    ref = W.ref if isinstance(W, Weights) else C.byref(W)
+    _check(lib().fb_gemv_launch_plan(ref, batch, flags, sms, C.cast(out, C.c_void_p)), "fb_gemv_launch_plan")
+    return dict(zip(("C", "cpb", "RB", "warps", "smem", "V"), list(out)))
+
+
+def fb_device_errors(clear: bool = True) -> int:
+    """Error bits raised by GEMV kernels since the last clear (synchronises the device)."""
+    flags = C.c_uint(0)
+    _check(lib().fb_device_errors(C.cast(C.byref(flags), C.c_void_p), int(clear)), "fb_device_errors")
+    return flags.value

@@ -6,36 +6,35 @@
 //
 // Work units.  A "virtual panel" is one panel (<= 256 columns) of one base,
 // global or salient; the matrix has V of them.  Rows come in chunks of 32,
-// one row per lane.  A thread-block cluster of C CTAs owns one block of cpb
+// one row per lane; an "item" is one chunk of one virtual panel (32 rows x
+// <= 32 bytes).  A thread-block cluster of C CTAs owns one block of cpb
 // chunks; CTA j of the cluster takes a contiguous, balanced slice of the V
 // virtual panels, so the cluster covers every column of its rows.
 //
-// Per CTA:
-//   1. before the programmatic-launch wait: the first weight words of every
-//      warp (128-bit, read-only, no L1 allocation) and their row scales, and
-//      the column scales and salient indices of the first table group;
-//   2. after the wait (or before it, for calls flagged independent): x, then
-//      z = alpha_c * x for the group's columns (column scales fused: LUT-BSF;
-//      salient panels read x[s_idx[t]] -- the virtual columnar mapping), and
-//      the group's tables in shared memory;
-//   3. each lane walks its row's bytes: one `prmt` merges a weight byte and
+// Per CTA (8 warps; warp w owns chunks w, w+8, ... of the row block):
+//   1. before the programmatic-launch wait: the first weight items of every
+//      warp start streaming into the warp's ring of shared-memory slots (one
+//      bulk asynchronous copy per item, completion on an mbarrier), and the
+//      row scales of the row block are staged in shared memory;
+//   2. per panel, all 256 threads build its byte tables in shared memory
+//      (LUT-BSF: z = alpha_c * x, salient panels reading x[s_idx[t]] -- the
+//      virtual columnar mapping -- and for each group of 8 columns the 256
+//      sums sum_t (bit t of b ? +z_t : -z_t), each the sum of the two 4-column
+//      tables of its nibbles), double-buffered, one CTA barrier per panel;
+//   3. each lane walks its row's 32 bytes: one `prmt` merges a weight byte and
 //      the lane's column offset into a table address, one shared load fetches
 //      the partial sum, packed fp32x2 adds accumulate (a gather-add, no tensor
-//      cores); the sum of each panel is scaled by alpha_r once (alpha_r applied
-//      in the reduction) and added to the row's partial;
-//   4. the cluster synchronises and each CTA sums the C partials of its share
-//      of the rows from distributed shared memory, in a fixed order, and
-//      writes y.  No workspace, no atomics, no spin-waits; deterministic.
+//      cores); each item's sum is scaled by alpha_r once (alpha_r applied in
+//      the reduction) and added to the row's partial;
+//   4. each CTA pushes its row partials into the shared memory of the CTA
+//      that owns those rows, the cluster synchronises once, and each owner
+//      sums its C inbox slots in rank order and writes y.  No workspace, no
+//      atomics; deterministic.
 //
-// Shared-memory tables of one virtual panel (byte offsets, q = byte group of
-// the panel, entries fp32):
-//   g = 8: T[p][q] at p*256 + 4q; two panels share a 64 KiB region, the second
-//          at +128 (p < 256)
-//   g = 4: low nibble T[v][q] at v*256 + 4q, high nibble at v*256 + 128 + 4q
-//   g = 2: T[s][v][q] at ((s << 2) + v)*128 + 4q (s: 2-bit field of the byte)
-//   g = 1: T[s][v][q] at ((s << 1) + v)*128 + 4q
-// Lane l at stored position u reads byte group (l+u) mod Bp (the rotation of
-// the packed layout), so a warp's 32 lookups hit 32 different banks.
+// Byte tables: entry b of byte group q (columns 8q .. 8q+7 of the panel) is
+// at b*256 + 4q bytes; the two buffers interleave, the second at +128.  Lane
+// l at stored position u reads byte group (l+u) mod Bp (the rotation of the
+// packed layout), so a warp's 32 lookups hit 32 different banks.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -43,6 +42,8 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 #include <new>
 
 #include "fb_internal.cuh"
@@ -53,11 +54,12 @@ namespace fb {
 namespace {
 
 constexpr int kMaxCluster = 8;
-constexpr int kThreads = 256;           // 8 warps; thread t stages column t of a panel
-constexpr int kWarps = kThreads / 32;
-constexpr int kRing = 4;                // weight items per warp in flight ahead of use
-constexpr int kMaxGroup = 8;            // virtual panels per table group
-constexpr int kMaxCpb = 64;             // chunks per row block
+constexpr int kNW = 8;                  // warps per CTA
+constexpr int kMaxCpb = 16;             // chunks per row block (two per warp)
+constexpr size_t kMaxDynSmem = 200 * 1024;   // dynamic shared memory per CTA
+constexpr double kOverlapDepth = 8;          // launches in flight together, for the planner
+constexpr size_t kSmemPerSM = 228 * 1024;
+constexpr size_t kStaticSmem = 1024;          // the kernel's static shared memory, rounded up
 constexpr unsigned kKnownFlags = FB_GEMV_PDL | FB_GEMV_INDEPENDENT;
 
 struct GemvArgs {
@@ -72,35 +74,72 @@ struct GemvArgs {
     float *y;
     int M, M_pad, N, K, nS, nS_pad, Ks;
     int Pg, Ps;
-    int nchunks, cpb, n_my;   // chunks per row block; per warp (cpb = warps * n_my)
-    int group_max;            // virtual panels per table group
+    int nchunks, cpb;         // chunks (32 rows) in the matrix, per row block
     int ldx, ldy;
     unsigned flags;
     int C;
     int vsplit[kMaxCluster + 1];   // CTA j of a cluster: virtual panels [vsplit[j], vsplit[j+1])
-    int first_sal[kMaxCluster], first_k[kMaxCluster], first_p[kMaxCluster];   // decoded vsplit[j]
-    int narrow_mask[kMaxCluster];  // bit 0: rank j has the narrow global tail panel; bit 1: a narrow salient one
 };
-
-// Table bytes per virtual panel slot in a group.
-__host__ __device__ constexpr int table_stride(int g) { return g == 8 ? 32768 : g == 4 ? 4096 : 2048; }
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-__device__ __forceinline__ uint4 ld_stream16(const void *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
+// ---- bulk asynchronous copies into shared memory, signalled on mbarriers ----
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
 }
-__device__ __forceinline__ uint32_t ld_stream4(const void *p) {
-    uint32_t r;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
-    return r;
+__device__ __forceinline__ void mbar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// One copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
+// global memory into this CTA's shared memory; the barrier's phase completes
+// when the bytes have landed.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%2], %1;\n\t"
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%3], %1, [%2];\n\t}"
+        ::"r"(dst), "r"(bytes), "r"(bar), "l"(src)
+        : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for a barrier phase: gives up after kWaitLimitNs (or
+// kWaitLimitIters polls) and returns false.
+constexpr unsigned long long kWaitLimitNs = 200ull * 1000 * 1000;
+constexpr int kWaitLimitIters = 1 << 24;
+__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    unsigned long long t0 = 0;
+    for (int it = 0; it < kWaitLimitIters; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31) == 31) {
+            const unsigned long long now = global_ns();
+            if (t0 == 0)
+                t0 = now;
+            else if (now - t0 > kWaitLimitNs)
+                return false;
+        }
+    }
+    return false;
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -157,15 +196,6 @@ __device__ __forceinline__ float x_value(uint32_t bits) {
     return __uint_as_float(bits << 16);
 }
 
-// sum_{t<4} (bit t of a ? +1 : -1) * z_t, added in order t = 0..3.
-__device__ __forceinline__ float sum4(float z0, float z1, float z2, float z3, int a) {
-    float s = (a & 1) ? z0 : -z0;
-    s = __fadd_rn(s, (a & 2) ? z1 : -z1);
-    s = __fadd_rn(s, (a & 4) ? z2 : -z2);
-    s = __fadd_rn(s, (a & 8) ? z3 : -z3);
-    return s;
-}
-
 // The 16 entries sum_{t<4} (bit t of a ? +1 : -1) * z_t, a = 0..15, as
 // (+-z0 +- z1) + (+-z2 +- z3).
 __device__ __forceinline__ void sums16(float z0, float z1, float z2, float z3, float (&e)[16]) {
@@ -175,51 +205,53 @@ __device__ __forceinline__ void sums16(float z0, float z1, float z2, float z3, f
     for (int a = 0; a < 16; ++a) e[a] = __fadd_rn(p01[a & 3], p23[a >> 2]);
 }
 
-// One virtual panel: where its words and row scales live, its width.
+// One virtual panel: where its words live, its width and its scales.
 struct VPanel {
     const uint8_t *pl;   // chunk block 0 of this panel and base
-    const float *ar;     // row scales of this base
     const float *ac;     // column scales of this base, or null (all ones)
     int col0;            // first column of the panel (global, or compact salient)
     int Bp;              // byte groups (width / 8)
-    int k, p, sal;       // base, panel, 1 for salient panels
+    int kb;              // row-scale base: k for global panels, K + k for salient ones
+    int sal;             // 1 for salient panels
 };
 
-__device__ __forceinline__ void vp_set(const GemvArgs &a, VPanel &r, int sal, int k, int p) {
-    const int ncols = sal ? a.nS_pad : a.N;
-    r.sal = sal;
-    r.k = k;
-    r.p = p;
-    r.col0 = p * kPanelCols;
-    r.Bp = panel_width(ncols, p) >> 3;
-    r.pl = (sal ? a.s_planes : a.planes) + (size_t)k * a.M_pad * (size_t)(ncols / 8) + (size_t)32 * p * a.M_pad;
-    r.ar = (sal ? a.s_alpha_r : a.alpha_r) + (size_t)k * a.M;
-    r.ac = sal ? a.s_alpha_c + (size_t)k * a.nS : (a.alpha_c ? a.alpha_c + (size_t)k * a.N : nullptr);
-}
+// Position of a virtual panel in the order global panels of base 0, 1, ...
+// then salient ones; a CTA walks its slice one panel at a time.
+struct PanelPos {
+    int sal, k, p;
+};
 
-// Virtual panel v: global panels of base 0, 1, ... then salient ones.
-__device__ __forceinline__ void vp_first(const GemvArgs &a, VPanel &r, int v) {
+__device__ __forceinline__ PanelPos panel_pos(const GemvArgs &a, int v) {
     const int ng = a.Pg * a.K;
-    if (v < ng) {
-        const int k = v / a.Pg;
-        vp_set(a, r, 0, k, v - k * a.Pg);
-    } else {
-        const int k = (v - ng) / max(a.Ps, 1);
-        vp_set(a, r, 1, k, (v - ng) - k * a.Ps);
-    }
+    PanelPos q;
+    q.sal = v >= ng;
+    const int r = q.sal ? v - ng : v, P = q.sal ? max(a.Ps, 1) : a.Pg;
+    q.k = r / P;
+    q.p = r - q.k * P;
+    return q;
 }
 
-// The virtual panel after r, without a division.
-__device__ __forceinline__ void vp_next(const GemvArgs &a, VPanel &r) {
-    int sal = r.sal, k = r.k, p = r.p + 1;
-    if (p == (sal ? a.Ps : a.Pg)) {
-        p = 0;
-        if (++k == (sal ? a.Ks : a.K) && !sal) {
-            sal = 1;
-            k = 0;
+__device__ __forceinline__ void panel_next(const GemvArgs &a, PanelPos &q) {
+    if (++q.p == (q.sal ? a.Ps : a.Pg)) {
+        q.p = 0;
+        if (++q.k == (q.sal ? a.Ks : a.K)) {
+            q.sal = 1;
+            q.k = 0;
         }
     }
-    vp_set(a, r, sal, k, p);
+}
+
+__device__ __forceinline__ VPanel panel_at(const GemvArgs &a, const PanelPos &q) {
+    const int ncols = q.sal ? a.nS_pad : a.N;
+    VPanel r;
+    r.sal = q.sal;
+    r.kb = q.sal ? a.K + q.k : q.k;
+    r.col0 = q.p * kPanelCols;
+    r.Bp = panel_width(ncols, q.p) >> 3;
+    r.pl = (q.sal ? a.s_planes : a.planes) + (size_t)q.k * a.M_pad * (size_t)(ncols / 8) +
+           (size_t)32 * q.p * a.M_pad;
+    r.ac = q.sal ? a.s_alpha_c + (size_t)q.k * a.nS : (a.alpha_c ? a.alpha_c + (size_t)q.k * a.N : nullptr);
+    return r;
 }
 
 // Column c of a panel: its scale alpha_c and the column of x it reads (-1:
@@ -231,38 +263,16 @@ __device__ __forceinline__ void column_source(const GemvArgs &a, const VPanel &v
     if (c >= vp.Bp * 8) return;
     const int col = vp.col0 + c;
     if (!vp.sal) {
-        ac = vp.ac ? __ldg(vp.ac + col) : 1.0f;
         xi = col;
+        if (vp.ac)
+            ac = __ldg(vp.ac + col);
+        else
+            ac = 1.0f;
     } else if (col < a.nS) {
         ac = __ldg(vp.ac + col);
         const uint32_t jx = __ldg(a.s_idx + col);
         xi = jx < (uint32_t)a.N ? (int)jx : -1;   // an invalid index contributes 0
     }
-}
-
-// The row's words of one chunk of one panel; positions past a narrow
-// panel's Bp bytes are zero.
-__device__ __forceinline__ void load_item(const VPanel &vp, int c, const GemvArgs &a, int lane, uint32_t (&w)[8],
-                                          float &arv) {
-#pragma unroll
-    for (int m = 0; m < 8; ++m) w[m] = 0;
-    arv = 0.0f;
-    if (c >= a.nchunks) return;   // padding chunk of the last row block
-    const uint8_t *blk = vp.pl + (size_t)32 * vp.Bp * c;
-    if (vp.Bp == 32) {
-        const uint4 x0 = ld_stream16(blk + 16 * lane), x1 = ld_stream16(blk + 512 + 16 * lane);
-        w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
-        w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
-    } else if (vp.Bp == 16) {
-        const uint4 x0 = ld_stream16(blk + 16 * lane);
-        w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
-    } else {
-#pragma unroll
-        for (int m = 0; m < 7; ++m)
-            if (m < vp.Bp / 4) w[m] = ld_stream4(blk + 128 * m + 4 * lane);
-    }
-    const int row = c * kChunkRows + lane;
-    arv = row < a.M ? __ldg(vp.ar + row) : 0.0f;
 }
 
 // Column offsets of a full panel: byte j of offp[m] = 4 * ((lane + 4m + j) mod 32).
@@ -275,330 +285,323 @@ __device__ __forceinline__ void full_offsets(int lane, uint32_t (&offp)[8]) {
     }
 }
 
-// Column offsets of a narrow panel (Bp < 32), one word (8 per lane) per
-// call: byte j of word m = 4 * ((lane + u) mod Bp) for u = 4m + j < Bp, and
-// column 31 (built all zero) for the positions past Bp.
-__device__ __forceinline__ uint32_t narrow_offset_word(int lane, int m, int Bp) {
-    uint32_t o = 0;
+// Column offsets of a narrow panel (Bp < 32): byte j of word m = 4 * ((lane
+// + u) mod Bp) for u = 4m + j < Bp, and column 31 (built all zero) for the
+// positions past Bp.  Narrow panels are rare, so this stays out of line.
+struct Offsets {
+    uint32_t w[8];
+};
+__device__ __noinline__ Offsets narrow_offsets(int lane, int Bp) {
+    Offsets o;
+    const int r = lane % Bp;
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-        const int u = 4 * m + jj;
-        const int q = u < Bp ? (lane + u) % Bp : 31;
-        o |= (uint32_t)(4 * q) << (8 * jj);
+    for (int m = 0; m < 8; ++m) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int u = 4 * m + jj;
+            int q = r + u;
+            q = q >= Bp ? q - Bp : q;
+            q = u < Bp ? q : 31;
+            word |= (uint32_t)(4 * q) << (8 * jj);
+        }
+        o.w[m] = word;
     }
     return o;
 }
 
-// Sum of the table entries selected by one row's 32 stored bytes.  w holds
-// position u in byte u%4 of w[u/4]; offp holds, in the same places, the byte
-// offset 4*q of the column each position maps to.
-template <int G>
+// Sum of the byte-table entries selected by one row's 32 stored bytes.  w
+// holds position u in byte u%4 of w[u/4]; offp holds, in the same places,
+// the byte offset 4*q of the column group each position maps to.
 __device__ __forceinline__ float lookup_row(const uint32_t (&w)[8], const uint32_t (&offp)[8], const float *tbl) {
-    unsigned long long acc0 = 0, acc1 = 0;
+    unsigned long long acc[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
-        if (G == 8) {
-            const float v0 = lds(tbl, prmt(w[m], offp[m], addr_sel(0)));
-            const float v1 = lds(tbl, prmt(w[m], offp[m], addr_sel(1)));
-            const float v2 = lds(tbl, prmt(w[m], offp[m], addr_sel(2)));
-            const float v3 = lds(tbl, prmt(w[m], offp[m], addr_sel(3)));
-            acc0 = fadd2(acc0, f2pack(v0, v1));
-            acc1 = fadd2(acc1, f2pack(v2, v3));
-        } else if (G == 4) {
-            const uint32_t w4 = w[m] >> 4;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const float lo = lds(tbl, prmt(w[m], offp[m], addr_sel(jj)) & 0x0FFFu);
-                const float hi = lds(tbl + 32, prmt(w4, offp[m], addr_sel(jj)) & 0x0FFFu);
-                if (jj & 1)
-                    acc1 = fadd2(acc1, f2pack(lo, hi));
-                else
-                    acc0 = fadd2(acc0, f2pack(lo, hi));
-            }
-        } else {
-            constexpr int kFields = 8 / G, kMask = (1 << G) - 1;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t byte = (w[m] >> (8 * jj)) & 0xFFu;
-                const uint32_t off = (offp[m] >> (8 * jj)) & 0xFFu;
-#pragma unroll
-                for (int s = 0; s < kFields; s += 2) {
-                    const uint32_t v0 = (byte >> (G * s)) & kMask, v1 = (byte >> (G * (s + 1))) & kMask;
-                    const float e0 = lds(tbl, (((uint32_t)s << G) + v0) * 128u + off);
-                    const float e1 = lds(tbl, (((uint32_t)(s + 1) << G) + v1) * 128u + off);
-                    acc0 = fadd2(acc0, f2pack(e0, e1));
-                }
-            }
-        }
+        const float v0 = lds(tbl, prmt(w[m], offp[m], addr_sel(0)));
+        const float v1 = lds(tbl, prmt(w[m], offp[m], addr_sel(1)));
+        const float v2 = lds(tbl, prmt(w[m], offp[m], addr_sel(2)));
+        const float v3 = lds(tbl, prmt(w[m], offp[m], addr_sel(3)));
+        acc[(2 * m) & 3] = fadd2(acc[(2 * m) & 3], f2pack(v0, v1));
+        acc[(2 * m + 1) & 3] = fadd2(acc[(2 * m + 1) & 3], f2pack(v2, v3));
     }
-    return __fadd_rn(f2sum(acc0), f2sum(acc1));
+    return __fadd_rn(__fadd_rn(f2sum(acc[0]), f2sum(acc[1])), __fadd_rn(f2sum(acc[2]), f2sum(acc[3])));
 }
 
-template <int G>
-__device__ __forceinline__ const float *table_of(const float *tbl, int slot) {
-    if (G == 8) return tbl + (slot >> 1) * 16384 + (slot & 1) * 32;
-    return tbl + slot * (table_stride(G) / 4);
+// LUT-BSF for one virtual panel, built by the whole CTA: lane q builds byte
+// group q (columns 8q .. 8q+7, z in zp), warp w its entries b = 32w .. 32w+31:
+// entry b = T_lo[b & 15] + T_hi[b >> 4], where T_lo and T_hi are the 16-entry
+// tables of the group's low and high 4 columns, each (+-z0 +- z1) + (+-z2 +-
+// z3).  Columns past a narrow panel's width have z = 0, so their entries are
+// 0.  T points at the buffer (entry b of group q at T[b*64 + q]).
+__device__ __forceinline__ void build_byte_table(const float *zp, float *T, int warp, int lane) {
+    const float4 za = *reinterpret_cast<const float4 *>(zp + 8 * lane);
+    const float4 zb = *reinterpret_cast<const float4 *>(zp + 8 * lane + 4);
+    float lo[16];
+    sums16(za.x, za.y, za.z, za.w, lo);
+    float hi[2];
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+        const int h = 2 * warp + s2;
+        const float s01 = __fadd_rn((h & 1) ? zb.x : -zb.x, (h & 2) ? zb.y : -zb.y);
+        const float s23 = __fadd_rn((h & 4) ? zb.z : -zb.z, (h & 8) ? zb.w : -zb.w);
+        hi[s2] = __fadd_rn(s01, s23);
+    }
+    float *col = T + (32 * warp) * 64 + lane;
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+        for (int v = 0; v < 16; ++v) col[(16 * s2 + v) * 64] = __fadd_rn(lo[v], hi[s2]);
 }
 
-// LUT-BSF: the tables of one group of virtual panels from z = alpha_c * x
-// (z is 0 past a narrow panel's width, so those table columns are 0).
-// Tasks (slot, q, r): q = byte group (consecutive threads -> consecutive
-// banks), r = 0..15 a row group of the table.
-template <int G>
-__device__ __forceinline__ void build_group(float *tbl, const float *zbuf, int gsize, int tid, int nthreads) {
-    if (G == 4 || G == 8) {
-        // g = 4: task (slot, q, half) writes the 16 entries of one nibble table.
-        // g = 8: task (slot, q, hi) writes the 16 entries lo[a] + hi-sum[hi].
-        const int ntask = gsize * 32 * (G == 4 ? 2 : 16);
-        for (int t = tid; t < ntask; t += nthreads) {
-            const int q = t & 31;
-            const int r = G == 4 ? (t >> 5) & 1 : (t >> 5) & 15;
-            const int slot = G == 4 ? t >> 6 : t >> 9;
-            const float *z = zbuf + slot * 256 + 8 * q;
-            float *col = const_cast<float *>(table_of<G>(tbl, slot)) + q;
-            float e[16];
-            if (G == 4) {
-                const float4 zz = *reinterpret_cast<const float4 *>(z + 4 * r);
-                sums16(zz.x, zz.y, zz.z, zz.w, e);
+// Set (bit 0) when a kernel gave up waiting for a weight copy; the rows of
+// that CTA are then written as NaN.  Read and cleared by fb_device_errors.
+__device__ unsigned int g_error_flags;
+
+// The row's words of one item of a narrow panel (Bp < 32) from its slot
+// (the block's bytes in the packed layout); positions past Bp are zero.
+struct Words {
+    uint32_t w[8];
+};
+__device__ __noinline__ Words read_item_narrow(const uint8_t *slot, int Bp, int lane) {
+    Words r;
 #pragma unroll
-                for (int a = 0; a < 16; ++a) col[a * 64 + 32 * r] = e[a];
-            } else {
-                const float4 za = *reinterpret_cast<const float4 *>(z);
-                const float4 zb = *reinterpret_cast<const float4 *>(z + 4);
-                sums16(za.x, za.y, za.z, za.w, e);
-                float h[16];
-                sums16(zb.x, zb.y, zb.z, zb.w, h);
-                float hr = h[0];
+    for (int m = 0; m < 8; ++m) r.w[m] = 0;
+    if (Bp == 16) {
+        const uint4 x0 = *reinterpret_cast<const uint4 *>(slot + 16 * lane);
+        r.w[0] = x0.x; r.w[1] = x0.y; r.w[2] = x0.z; r.w[3] = x0.w;
+    } else {
 #pragma unroll
-                for (int a = 1; a < 16; ++a) hr = r == a ? h[a] : hr;
-#pragma unroll
-                for (int a = 0; a < 16; ++a) col[(r * 16 + a) * 64] = __fadd_rn(e[a], hr);
-            }
-        }
-        return;
+        for (int m = 0; m < 7; ++m)
+            if (m < Bp / 4) r.w[m] = *reinterpret_cast<const uint32_t *>(slot + 128 * m + 4 * lane);
     }
-    const int ntask = gsize * 32 * 16;
-    for (int t = tid; t < ntask; t += nthreads) {
-        const int q = t & 31, r = (t >> 5) & 15, slot = t >> 9;
-        const float *z = zbuf + slot * 256 + 8 * q;
-        const float4 za = *reinterpret_cast<const float4 *>(z);
-        const float4 zb = *reinterpret_cast<const float4 *>(z + 4);
-        float *col = const_cast<float *>(table_of<G>(tbl, slot)) + q;
-        if (G == 2) {
-            const int s = r >> 2, v = r & 3;
-            const float lo0 = s == 0 ? za.x : s == 1 ? za.z : s == 2 ? zb.x : zb.z;
-            const float lo1 = s == 0 ? za.y : s == 1 ? za.w : s == 2 ? zb.y : zb.w;
-            float e = (v & 1) ? lo0 : -lo0;
-            e = __fadd_rn(e, (v & 2) ? lo1 : -lo1);
-            col[r * 32] = e;
-        } else {
-            const int s = r >> 1, v = r & 1;
-            const float zs = s == 0 ? za.x : s == 1 ? za.y : s == 2 ? za.z : s == 3 ? za.w
-                           : s == 4 ? zb.x : s == 5 ? zb.y : s == 6 ? zb.z : zb.w;
-            col[r * 32] = v ? zs : -zs;
-        }
-    }
+    return r;
 }
 
-template <int G, int XT>
-__global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
-    extern __shared__ __align__(16) float smem_f[];
-    // offsets of the (at most two) narrow panel widths: global tail, salient tail
-    __shared__ __align__(16) uint32_t s_noff[2][32][8];
+// The row's words of one item of a full panel from its slot.
+__device__ __forceinline__ void read_item_full(const uint8_t *slot, int lane, uint32_t (&w)[8]) {
+    const uint4 x0 = *reinterpret_cast<const uint4 *>(slot + 16 * lane);
+    const uint4 x1 = *reinterpret_cast<const uint4 *>(slot + 512 + 16 * lane);
+    w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
+    w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
+}
+
+// Shared-memory layout of one CTA (bytes): two interleaved byte tables |
+// z of two panels | two weight slots | row scales [KB][R] | row partials [R]
+// | cluster inbox.
+constexpr int kTableBytes = 65536;
+constexpr int kZBytes = 2 * kPanelCols * 4;
+constexpr int kSlotBytes = kMaxCpb * 1024;   // one panel of a row block: cpb blocks of <= 1 KiB
+constexpr int kItemsPerWarp = kMaxCpb / kNW;
+
+template <int XT>
+__global__ void __launch_bounds__(kNW * 32, 2) gemv_kernel(const __grid_constant__ GemvArgs args) {
+    extern __shared__ __align__(128) float smem_f[];
+    __shared__ __align__(8) unsigned long long s_bar[2];
+    // The launch's parameter block is new to every SM's constant cache, and the
+    // kernel would touch its fields one after another, each a miss; one
+    // parallel copy into shared memory pays that latency once.
+    __shared__ __align__(16) GemvArgs s_args;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    static_assert(sizeof(GemvArgs) % 4 == 0, "parameter block copied as words");
+    for (int i = tid; i < (int)(sizeof(GemvArgs) / 4); i += blockDim.x)
+        reinterpret_cast<int *>(&s_args)[i] = reinterpret_cast<const int *>(&args)[i];
+    if (tid == 0) {
+        mbar_init(smem_addr(&s_bar[0]));
+        mbar_init(smem_addr(&s_bar[1]));
+        mbar_init_fence();
+    }
+    __syncthreads();
+    const GemvArgs &a = s_args;
     cg::cluster_group cluster = cg::this_cluster();
     const int j = (int)cluster.block_rank();
     const int rb = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-    const int vb = a.vsplit[j], nv = a.vsplit[j + 1] - vb;
-    const int GM = a.group_max;
-    const int ngroups = (nv + GM - 1) / GM;
-    float *tbl = smem_f;
-    const int tfloats = G == 8 ? ((GM + 1) / 2) * 16384 : GM * (table_stride(G) / 4);
-    float *zbuf = tbl + tfloats;
-    float *part = zbuf + GM * 256;
+    const int vb = a.vsplit[j], n_v = a.vsplit[j + 1] - a.vsplit[j];
+    const int cpb = a.cpb, R = cpb * kChunkRows;
+    const int c_first = rb * cpb;
+    const int nvalid = min(cpb, a.nchunks - c_first);   // chunks of this row block inside the matrix
+    const int KB = a.K + a.Ks;                          // bases with row scales: global, then salient
     const bool independent = (a.flags & FB_GEMV_INDEPENDENT) != 0;
-    const int c_first = rb * a.cpb;   // first chunk of the row block
-    const int n_my = a.n_my;          // chunks per warp: c_first + warp + 8 * ci
     const size_t xoff = (size_t)b * a.ldx;
-    const int bp_gtail = panel_width(a.N, a.Pg - 1) >> 3;
-    const int bp_stail = a.Ps > 0 ? panel_width(a.nS_pad, a.Ps - 1) >> 3 : 32;
 
-    // ---- 1. weights and first-group column data, before the wait ----------
-    // Every warp walks the same padded item sequence: per table group, its
-    // real items (panel-major, n_my chunks each) padded to a multiple of kRing.
-    uint32_t ring[kRing][8];
-    float ring_ar[kRing];
-    int p_g = 0, p_pos = 0, p_ci = 0, p_vi = 0;   // producer: group, padded position, chunk, panel
-    VPanel p_vp;
-    vp_set(a, p_vp, a.first_sal[j], a.first_k[j], a.first_p[j]);
-    auto produce = [&](uint32_t (&w)[8], float &arv) {
-        if (p_g >= ngroups) return;
-        const int n_real = n_my * min(GM, nv - p_g * GM);
-        if (p_pos < n_real) {
-            load_item(p_vp, c_first + warp + kWarps * p_ci, a, lane, w, arv);
-            if (++p_ci == n_my) {
-                p_ci = 0;
-                if (++p_vi < nv) vp_next(a, p_vp);
-            }
-        }
-        if (++p_pos == (n_real + kRing - 1) / kRing * kRing) {
-            p_pos = 0;
-            ++p_g;
-        }
-    };
-#pragma unroll
-    for (int s = 0; s < kRing; ++s) produce(ring[s], ring_ar[s]);
+    float *tables = smem_f;
+    float *zbuf = smem_f + kTableBytes / 4;
+    uint8_t *slots = reinterpret_cast<uint8_t *>(smem_f) + kTableBytes + kZBytes;
+    float *s_ar = smem_f + (kTableBytes + kZBytes + 2 * kSlotBytes) / 4;
+    float *pw = s_ar + KB * R;
+    float *part = pw + R;
+    const uint32_t slots_s = smem_addr(slots), bar_s = smem_addr(&s_bar[0]);
 
-    // column data of a table group: thread t stages column t of each panel
-    float z_ac[kMaxGroup];
-    uint32_t z_x[kMaxGroup];
-    int z_xi[kMaxGroup];
-    auto stage_group = [&](int g0, bool read_x) {
-        const int gsize = min(GM, nv - g0);
-        VPanel vp;
-        if (g0 == 0)
-            vp_set(a, vp, a.first_sal[j], a.first_k[j], a.first_p[j]);
-        else
-            vp_first(a, vp, vb + g0);
-#pragma unroll
-        for (int gi = 0; gi < kMaxGroup; ++gi) {
-            z_ac[gi] = 0.0f;
-            z_xi[gi] = -1;
-            z_x[gi] = 0;
-            if (gi < gsize) {
-                if (gi > 0) vp_next(a, vp);
-                column_source(a, vp, tid, z_ac[gi], z_xi[gi]);
-                if (read_x && z_xi[gi] >= 0) z_x[gi] = load_x_bits<XT>(a.x, xoff + z_xi[gi]);
-            }
-        }
+    // ---- 1. weight copies and row scales, before the wait -------------------
+    // Panel vi's blocks of this row block are contiguous: one bulk copy into
+    // slot vi % 2, issued by thread 0.
+    uint32_t pending = 0, pend_par = 0;   // thread 0: slots with a copy in flight, its phase parity
+    auto issue = [&](int vi, const VPanel &vp) {
+        const uint32_t blk = 32u * (uint32_t)vp.Bp;
+        bulk_load(slots_s + (vi & 1) * kSlotBytes, vp.pl + (size_t)blk * c_first, blk * (uint32_t)nvalid,
+                  bar_s + 8 * (vi & 1));
+        pending |= 1u << (vi & 1);
+        pend_par = (pend_par & ~(1u << (vi & 1))) | ((uint32_t)(vi >> 1) & 1u) << (vi & 1);
     };
-#pragma unroll
-    for (int gi = 0; gi < kMaxGroup; ++gi) {
-        z_ac[gi] = 0.0f;
-        z_x[gi] = 0;
-        z_xi[gi] = -1;
-    }
-    if (nv > 0) stage_group(0, independent);
+    PanelPos pos_cur = panel_pos(a, vb), pos_ahead = pos_cur;   // panels vi and vi + 2
+    if (n_v > 0 && tid == 0) issue(0, panel_at(a, pos_ahead));
+    panel_next(a, pos_ahead);
+    if (n_v > 1 && tid == 0) issue(1, panel_at(a, pos_ahead));
+    panel_next(a, pos_ahead);
+
+    // column data of one panel: thread t stages column t
+    float z_ac = 0.0f;
+    uint32_t z_x = 0;
+    int z_xi = -1;
+    auto stage = [&](const VPanel &vp, bool read_x) {
+        z_x = 0;
+        column_source(a, vp, tid, z_ac, z_xi);
+        if (read_x && z_xi >= 0) z_x = load_x_bits<XT>(a.x, xoff + z_xi);
+    };
+    if (n_v > 0) stage(panel_at(a, pos_cur), independent);
     griddep_launch_dependents();
-    const int nmask = a.narrow_mask[j];
-    if (nmask) {
-        for (int t = tid; t < 2 * 32 * 8; t += kThreads) {
-            const int which = t >> 8, ln = (t >> 3) & 31, m = t & 7;
-            if (nmask & (1 << which)) s_noff[which][ln][m] = narrow_offset_word(ln, m, which == 0 ? bp_gtail : bp_stail);
-        }
+    // the row block's row scales, every base (rows past M: 0)
+    for (int t = tid; t < KB * R; t += blockDim.x) {
+        const int kb = t / R, r = t - kb * R, row = c_first * kChunkRows + r;
+        const float *src = kb < a.K ? a.alpha_r + (size_t)kb * a.M : a.s_alpha_r + (size_t)(kb - a.K) * a.M;
+        s_ar[t] = row < a.M ? __ldg(src + row) : 0.0f;
     }
 
     // ---- 2. activations (may be the previous kernel's output) --------------
     if (!independent) {
         griddep_wait();
-#pragma unroll
-        for (int gi = 0; gi < kMaxGroup; ++gi)
-            if (z_xi[gi] >= 0) z_x[gi] = load_x_bits<XT>(a.x, xoff + z_xi[gi]);
+        if (z_xi >= 0) z_x = load_x_bits<XT>(a.x, xoff + z_xi);
     }
+    zbuf[tid] = z_xi >= 0 ? __fmul_rn(z_ac, x_value<XT>(z_x)) : 0.0f;
+    if (n_v > 1) {
+        PanelPos p1 = pos_cur;
+        panel_next(a, p1);
+        stage(panel_at(a, p1), true);
+    }
+    __syncthreads();   // z of panel 0 and row scales written
 
-    // ---- 3. table groups and the item loop ----------------------------------
-    VPanel c_vp;                 // consumer: current panel, its chunk index
-    vp_set(a, c_vp, a.first_sal[j], a.first_k[j], a.first_p[j]);
-    int c_vi = 0, c_ci = 0;
-    uint32_t offp[8];
-    bool narrow = false;
-    float acc1 = 0.0f;           // the row's sum when each warp owns one chunk
+    // column offsets of a full panel (narrow panels compute theirs)
+    uint32_t off_full[8];
+    full_offsets(lane, off_full);
 
-    for (int g = 0; g < ngroups; ++g) {
-        const int g0 = g * GM, gsize = min(GM, nv - g0);
-        __syncthreads();   // the previous group's tables are no longer read
+    // ---- 3. per panel: its byte tables, then this warp's chunks -------------
+    // Warp w owns chunks w and w + 8 of the row block; each lane keeps its
+    // two rows' partial sums and current row scales in registers.  The words
+    // move to registers before the panel's barrier, so right after it the
+    // slot can take the panel two ahead.
+    bool failed = false;
+    float racc[kItemsPerWarp], rar[kItemsPerWarp];
 #pragma unroll
-        for (int gi = 0; gi < kMaxGroup; ++gi)
-            if (gi < gsize) zbuf[gi * 256 + tid] = z_xi[gi] >= 0 ? __fmul_rn(z_ac[gi], x_value<XT>(z_x[gi])) : 0.0f;
-        __syncthreads();
-        build_group<G>(tbl, zbuf, gsize, tid, kThreads);
-        if (g + 1 < ngroups) stage_group(g0 + GM, true);   // x is readable by now
-        __syncthreads();
-        if (g == 0) {                                      // offsets of the first panel
-            narrow = c_vp.Bp != 32;
-            if (narrow) {
-                const int which = c_vp.sal;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) offp[m] = s_noff[which][lane][m];
-            } else {
-                full_offsets(lane, offp);
-            }
+    for (int it = 0; it < kItemsPerWarp; ++it) racc[it] = rar[it] = 0.0f;
+    int kb_cur = -1;
+#pragma unroll 1
+    for (int vi = 0; vi < n_v; ++vi) {
+        const int buf = vi & 1;
+        const VPanel vp = panel_at(a, pos_cur);
+        const int Bp = vp.Bp;
+        uint32_t w[kItemsPerWarp][8];
+        bool ok = !failed;
+        if (ok) {
+            const uint32_t par = (uint32_t)(vi >> 1) & 1u;
+            ok = mbar_try_wait(bar_s + 8 * buf, par) || mbar_wait_bounded(bar_s + 8 * buf, par);
         }
-
-        const int n_real = n_my * gsize;
-        const int n_pad = (n_real + kRing - 1) / kRing * kRing;
-        for (int i0 = 0; i0 < n_pad; i0 += kRing) {
+        if (tid == 0 && ok) pending &= ~(1u << buf);
+        const uint8_t *slot = slots + buf * kSlotBytes;
 #pragma unroll
-            for (int s = 0; s < kRing; ++s) {
-                if (i0 + s < n_real) {
-                    const float sum = lookup_row<G>(ring[s], offp, table_of<G>(tbl, c_vi - g0));
-                    const float val = __fmul_rn(ring_ar[s], sum);
-                    if (n_my == 1) {
-                        acc1 = c_vi == 0 ? val : __fadd_rn(acc1, val);
-                    } else {
-                        float &pr = part[(warp + kWarps * c_ci) * kChunkRows + lane];
-                        pr = c_vi == 0 ? val : __fadd_rn(pr, val);
-                    }
-                    if (++c_ci == n_my) {
-                        c_ci = 0;
-                        if (++c_vi < nv) {
-                            vp_next(a, c_vp);
-                            if (c_vp.Bp != 32) {
-                                const int which = c_vp.sal;
+        for (int it = 0; it < kItemsPerWarp; ++it) {
+            const int cl = warp + kNW * it;
 #pragma unroll
-                                for (int m = 0; m < 8; ++m) offp[m] = s_noff[which][lane][m];
-                                narrow = true;
-                            } else if (narrow) {
-                                full_offsets(lane, offp);
-                                narrow = false;
-                            }
-                        }
-                    }
+            for (int m = 0; m < 8; ++m) w[it][m] = 0;
+            if (ok && cl < nvalid) {
+                if (Bp == 32) {
+                    read_item_full(slot + cl * 1024, lane, w[it]);
+                } else {
+                    const Words r = read_item_narrow(slot + cl * 32 * Bp, Bp, lane);
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) w[it][m] = r.w[m];
                 }
-                produce(ring[s], ring_ar[s]);   // the item kRing positions ahead
             }
         }
+        float *tb = tables + 32 * buf;
+        build_byte_table(zbuf + buf * kPanelCols, tb, warp, lane);
+        if (vi + 1 < n_v) {   // z of the next panel into the other buffer
+            zbuf[(buf ^ 1) * kPanelCols + tid] = z_xi >= 0 ? __fmul_rn(z_ac, x_value<XT>(z_x)) : 0.0f;
+        }
+        VPanel vp2;
+        if (vi + 2 < n_v) {
+            vp2 = panel_at(a, pos_ahead);
+            stage(vp2, true);
+        }
+        panel_next(a, pos_cur);
+        panel_next(a, pos_ahead);
+        // tables of panel vi complete, the slot read, the other table's readers done
+        failed = __syncthreads_or(!ok) != 0;
+        if (failed) continue;
+        if (tid == 0 && vi + 2 < n_v) issue(vi + 2, vp2);
+        if (vp.kb != kb_cur) {   // a new base: its row scales
+            kb_cur = vp.kb;
+#pragma unroll
+            for (int it = 0; it < kItemsPerWarp; ++it) {
+                const int cl = warp + kNW * it;
+                if (cl < cpb) rar[it] = s_ar[kb_cur * R + cl * kChunkRows + lane];
+            }
+        }
+        uint32_t offp[8];
+        if (Bp == 32) {
+#pragma unroll
+            for (int m = 0; m < 8; ++m) offp[m] = off_full[m];
+        } else {
+            const Offsets o = narrow_offsets(lane, Bp);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) offp[m] = o.w[m];
+        }
+#pragma unroll
+        for (int it = 0; it < kItemsPerWarp; ++it) {
+            if (warp + kNW * it < nvalid) racc[it] = __fadd_rn(racc[it], __fmul_rn(rar[it], lookup_row(w[it], offp, tb)));
+        }
     }
-    if (n_my == 1) {
-        part[warp * kChunkRows + lane] = acc1;
-    } else if (nv == 0) {
-        for (int ci = 0; ci < n_my; ++ci) part[(warp + kWarps * ci) * kChunkRows + lane] = 0.0f;
+#pragma unroll
+    for (int it = 0; it < kItemsPerWarp; ++it) {
+        const int cl = warp + kNW * it;
+        if (cl < cpb) pw[cl * kChunkRows + lane] = racc[it];
+    }
+    if (failed && tid == 0) {
+        // Wait (bounded) for the copies still in flight, so none lands after
+        // the CTA has gone, then flag the failure.
+        for (int s2 = 0; s2 < 2; ++s2)
+            if (pending & (1u << s2)) mbar_wait_bounded(bar_s + 8 * s2, (pend_par >> s2) & 1u);
+        atomicOr(&g_error_flags, 1u);
     }
 
-    // ---- 4. cluster reduction of the row partials --------------------------
+    // ---- 4. the cluster's row partials, in a fixed order --------------------
+    // Rows are owned in runs of Rq: rank o sums rows [o*Rq, min((o+1)*Rq, R)).
+    // Every CTA pushes its row partials into the owner's inbox (slot = its
+    // own rank), one cluster barrier makes them visible, and each owner adds
+    // its inbox in rank order.  After the barrier no CTA touches another's
+    // shared memory, so none has to wait for the others before exiting.
+    const int Rq = (R + a.C - 1) / a.C;
+    __syncthreads();
+    for (int r = tid; r < R; r += blockDim.x) {
+        const float sum = failed ? __int_as_float(0x7fc00000) : pw[r];
+        const int owner = r / Rq;
+        float *inbox = cluster.map_shared_rank(part, owner);
+        inbox[j * Rq + (r - owner * Rq)] = sum;
+    }
     cluster.sync();
-    const int R = a.cpb * kChunkRows;
-    const int r_lo = (int)((long)R * j / a.C), r_hi = (int)((long)R * (j + 1) / a.C);
-    for (int r = r_lo + tid; r < r_hi; r += kThreads) {
-        float v[kMaxCluster];
-#pragma unroll
-        for (int jj = 0; jj < kMaxCluster; ++jj) v[jj] = jj < a.C ? cluster.map_shared_rank(part, jj)[r] : 0.0f;
-        float sum = v[0];
-#pragma unroll
-        for (int jj = 1; jj < kMaxCluster; ++jj)
-            if (jj < a.C) sum = __fadd_rn(sum, v[jj]);
+    for (int i = tid; i < Rq; i += blockDim.x) {
+        const int r = j * Rq + i;
+        if (r >= R) break;
+        float sum = part[i];
+        for (int jj = 1; jj < a.C; ++jj) sum = __fadd_rn(sum, part[jj * Rq + i]);
         const int row = c_first * kChunkRows + r;
         if (row < a.M) a.y[(size_t)b * a.ldy + row] = sum;
     }
-    cluster.sync();   // keep this CTA's partials alive until every reader is done
     if (independent) griddep_wait();   // complete only after the previous kernel
 }
 
 using KernelFn = void (*)(GemvArgs);
 
-template <int G>
-KernelFn pick_xt(fb_dtype t) {
-    return t == FB_F32 ? gemv_kernel<G, FB_F32> : t == FB_F16 ? gemv_kernel<G, FB_F16> : gemv_kernel<G, FB_BF16>;
-}
-
-KernelFn pick_kernel(int g, fb_dtype t) {
-    switch (g) {
-        case 8: return pick_xt<8>(t);
-        case 4: return pick_xt<4>(t);
-        case 2: return pick_xt<2>(t);
-        default: return pick_xt<1>(t);
-    }
+KernelFn pick_kernel(fb_dtype t) {
+    return t == FB_F32 ? gemv_kernel<FB_F32> : t == FB_F16 ? gemv_kernel<FB_F16> : gemv_kernel<FB_BF16>;
 }
 
 fb_status check_weights(const fb_weights *W) {
@@ -617,36 +620,44 @@ fb_status check_weights(const fb_weights *W) {
     return FB_OK;
 }
 
-// The launch plan: cluster size, split of the virtual panels over the
-// cluster, row block size.  Chosen by a cost model of the shared-memory pipe
-// (the binding resource): per CTA, lookups (rows x byte groups x 8/g) plus
-// table entries built, plus a fixed per-CTA cost; CTAs beyond one per SM form
-// further waves.
 struct Plan {
     int M_pad, Pg, Ps, nS_pad, V, nchunks;
-    int C, cpb, nwarps, n_my, RB, group_max;   // nwarps is always kWarps
+    int C, cpb, RB, nwarps;
     int vsplit[kMaxCluster + 1];
     size_t smem;
 };
 
 struct PlanKey {
     int M, N, K, g, nS, Ks, batch, sms;
+    bool independent;
     bool operator==(const PlanKey &o) const {
         return M == o.M && N == o.N && K == o.K && g == o.g && nS == o.nS && Ks == o.Ks && batch == o.batch &&
-               sms == o.sms;
+               sms == o.sms && independent == o.independent;
     }
 };
 
-// Every virtual panel costs one full 32-position lookup per row (narrow
-// panels look up zero columns past their width), so the split over the
-// cluster balances panel counts.
 void split_panels(int V, int C, int *vsplit, int *max_n) {
     *max_n = 0;
     for (int jj = 0; jj <= C; ++jj) vsplit[jj] = (int)((long)V * jj / C);
     for (int jj = 0; jj < C; ++jj) *max_n = std::max(*max_n, vsplit[jj + 1] - vsplit[jj]);
 }
 
-Plan make_plan(const fb_weights *W, int batch, int sms) {
+// Dynamic shared memory of a CTA with cpb chunks of rows and KB bases:
+// tables, z, rings, row scales, row partials and the inbox of row partials
+// pushed by the cluster (C * ceil(R / C) <= R + C floats).
+size_t smem_for(int cpb, int KB) {
+    const size_t R = (size_t)cpb * kChunkRows;
+    return (size_t)kTableBytes + kZBytes + 2 * (size_t)kSlotBytes + R * KB * 4 + R * 4 + (R + kMaxCluster) * 4;
+}
+
+// The launch plan: cluster size C (the split of the V virtual panels over
+// the cluster's CTAs) and row block size (cpb chunks of 32 rows).  Chosen
+// by a cost model in SM cycles.  Per panel a CTA writes 32 KiB of tables
+// (256 shared-memory store cycles) and, per chunk of its rows, reads 1 KiB
+// of weights through the shared-memory pipe and makes 32 table lookups
+// (48 cycles); latencies: a panel's build and barrier, an item per warp, a
+// fixed prologue and reduction.
+Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
     Plan pl;
     pl.M_pad = round_up(W->M, kChunkRows);
     pl.Pg = num_panels(W->N);
@@ -654,27 +665,39 @@ Plan make_plan(const fb_weights *W, int batch, int sms) {
     pl.Ps = W->nS > 0 ? num_panels(pl.nS_pad) : 0;
     pl.V = pl.Pg * W->K + pl.Ps * (W->nS > 0 ? W->Ks : 0);
     pl.nchunks = pl.M_pad / kChunkRows;
-    const int g = W->g;
-    const double lookups_per_item = 32.0 * 32.0 * 8.0 / g;   // one chunk of one panel
-    const double build_per_panel = g == 8 ? 8192 : g == 4 ? 1024 : 512;
-    const double fixed = 6000;   // prologue, syncs, reduce, in lookup units
+    pl.nwarps = kNW;
+    const int KB = W->K + (W->nS > 0 ? W->Ks : 0);
+    const double build_mio = 256, item_mio = 48;          // shared-memory pipe cycles
+    const double build_lat = 500, item_lat = 700, fixed = 4000;   // latency, cycles
     double best = 1e300;
-    pl.nwarps = kWarps;
     pl.C = 1;
-    pl.cpb = std::min(kMaxCpb, round_up(pl.nchunks, kWarps));
-    pl.RB = ceil_div(pl.nchunks, pl.cpb);
+    pl.cpb = 1;
+    pl.RB = pl.nchunks;
     pl.vsplit[0] = 0;
     pl.vsplit[1] = pl.V;
     for (int C = 1; C <= std::min(kMaxCluster, pl.V); ++C) {
-        int vs[kMaxCluster + 1], max_n;
-        split_panels(pl.V, C, vs, &max_n);
-        for (int cpb = kWarps; cpb <= kMaxCpb; cpb += kWarps) {
+        int vs[kMaxCluster + 1], nvm;
+        split_panels(pl.V, C, vs, &nvm);
+        for (int cpb = 1; cpb <= std::min(kMaxCpb, pl.nchunks); ++cpb) {
             const int RB = ceil_div(pl.nchunks, cpb);
-            if (RB > 65535) continue;   // grid.y limit
-            if (cpb > kWarps && ceil_div(pl.nchunks, cpb - kWarps) == RB) continue;   // same split, fewer rows
+            if (RB > 65535) continue;
+            if (cpb > 1 && ceil_div(pl.nchunks, cpb - 1) == RB) continue;   // same split, fewer rows
+            const size_t smem = smem_for(cpb, KB);
+            if (smem > kMaxDynSmem) continue;
+            const int occ = smem + kStaticSmem + 1024 <= kSmemPerSM / 2 ? 2 : 1;
             const long ctas = (long)C * RB * batch;
-            const double work = cpb * max_n * lookups_per_item / 32.0 + max_n * build_per_panel + fixed;
-            const double cost = (double)((ctas + sms - 1) / sms) * work;
+            const double mio = nvm * (build_mio + item_mio * cpb);   // per CTA
+            const double lat = fixed + nvm * (build_lat + std::ceil((double)cpb / kNW) * item_lat);
+            const double waves = std::ceil((double)ctas / ((double)sms * occ));
+            const double per_sm = std::ceil((double)ctas / sms) * mio;
+            // A dependent call is timed alone: its critical path counts.  Calls
+            // flagged independent overlap their neighbours, so what counts is
+            // the SM time they occupy, plus a share of one CTA's latency for
+            // the launches that do not overlap.
+            const double cost =
+                independent ? std::max((double)ctas * lat / ((double)sms * occ), (double)ctas * mio / sms) +
+                                  lat / kOverlapDepth
+                            : std::max(per_sm, waves * lat);
             if (cost < best * 0.999) {
                 best = cost;
                 pl.C = C;
@@ -684,26 +707,36 @@ Plan make_plan(const fb_weights *W, int batch, int sms) {
             }
         }
     }
-    pl.n_my = pl.cpb / kWarps;
-    pl.group_max = g == 8 ? 2 : kMaxGroup;
-    const size_t tbytes = g == 8 ? (size_t)((pl.group_max + 1) / 2) * 65536 : (size_t)pl.group_max * table_stride(g);
-    pl.smem = tbytes + (size_t)pl.group_max * 256 * 4 + (size_t)pl.cpb * kChunkRows * 4;
+    // Tuning aid: FB_PLAN="C,cpb" forces the cluster size and row block
+    // (clamped to what the matrix allows); read at each plan construction.
+    if (const char *ov = getenv("FB_PLAN")) {
+        int oc = 0, ocpb = 0;
+        if (sscanf(ov, "%d,%d", &oc, &ocpb) == 2 && oc >= 1 && ocpb >= 1) {
+            pl.C = std::min(std::min(oc, kMaxCluster), pl.V);
+            pl.cpb = std::min(std::min(ocpb, kMaxCpb), pl.nchunks);
+            while (pl.cpb > 1 && smem_for(pl.cpb, KB) > kMaxDynSmem) --pl.cpb;
+            pl.RB = ceil_div(pl.nchunks, pl.cpb);
+            int nvm;
+            split_panels(pl.V, pl.C, pl.vsplit, &nvm);
+        }
+    }
+    pl.smem = smem_for(pl.cpb, KB);
     return pl;
 }
 
-const Plan &cached_plan(const fb_weights *W, int batch, int sms) {
+const Plan &cached_plan(const fb_weights *W, int batch, int sms, bool independent) {
     struct Entry {
         PlanKey key;
         Plan plan;
     };
     thread_local Entry memo[16];
     thread_local int used = 0, next = 0;
-    const PlanKey key{W->M, W->N, W->K, W->g, W->nS, W->nS > 0 ? W->Ks : 0, batch, sms};
+    const PlanKey key{W->M, W->N, W->K, W->g, W->nS, W->nS > 0 ? W->Ks : 0, batch, sms, independent};
     for (int i = 0; i < used; ++i)
         if (memo[i].key == key) return memo[i].plan;
     Entry &e = memo[next];
     e.key = key;
-    e.plan = make_plan(W, batch, sms);
+    e.plan = make_plan(W, batch, sms, independent);
     next = (next + 1) % 16;
     used = std::min(used + 1, 16);
     return e.plan;
@@ -772,8 +805,8 @@ extern "C" fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtyp
         return FB_ERR_INVALID_VALUE;
     if (!aligned(X, es) || !aligned(Y, 4)) return FB_ERR_MISALIGNED;
 
-    const Plan &pl = cached_plan(W, batch, sm_count());
-    const KernelFn fn = pick_kernel(W->g, t);
+    const Plan &pl = cached_plan(W, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0);
+    const KernelFn fn = pick_kernel(t);
     if (!prepare_kernel(fn, pl.smem)) return FB_ERR_CUDA;
 
     GemvArgs a;
@@ -797,34 +830,11 @@ extern "C" fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtyp
     a.Ps = pl.Ps;
     a.nchunks = pl.nchunks;
     a.cpb = pl.cpb;
-    a.n_my = pl.n_my;
-    a.group_max = pl.group_max;
     a.ldx = ldx;
     a.ldy = ldy;
     a.flags = flags;
     a.C = pl.C;
     std::copy(pl.vsplit, pl.vsplit + kMaxCluster + 1, a.vsplit);
-    const int ng = pl.Pg * W->K;
-    const bool g_narrow = W->N % kPanelCols != 0, s_narrow = pl.nS_pad % kPanelCols != 0;
-    for (int jj = 0; jj < kMaxCluster; ++jj) {
-        a.first_sal[jj] = a.first_k[jj] = a.first_p[jj] = 0;
-        a.narrow_mask[jj] = 0;
-        if (jj >= pl.C) continue;
-        const int v0 = pl.vsplit[jj];
-        if (v0 < ng) {
-            a.first_k[jj] = v0 / pl.Pg;
-            a.first_p[jj] = v0 % pl.Pg;
-        } else if (pl.Ps > 0) {
-            a.first_sal[jj] = 1;
-            a.first_k[jj] = (v0 - ng) / pl.Ps;
-            a.first_p[jj] = (v0 - ng) % pl.Ps;
-        }
-        for (int v = pl.vsplit[jj]; v < pl.vsplit[jj + 1]; ++v) {
-            if (v < ng && g_narrow && v % pl.Pg == pl.Pg - 1) a.narrow_mask[jj] |= 1;
-            if (v >= ng && s_narrow && (v - ng) % pl.Ps == pl.Ps - 1) a.narrow_mask[jj] |= 2;
-        }
-    }
-
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.C, pl.RB, batch);
     cfg.blockDim = dim3(pl.nwarps * 32);
@@ -846,8 +856,32 @@ extern "C" fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtyp
     return status_of(cudaLaunchKernelEx(&cfg, fn, a));
 }
 
+extern "C" fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned flags, int sms, int *out) {
+    if (check_weights(W) != FB_OK || batch < 1 || batch > kMaxBatch || sms < 1 || !out || (flags & ~kKnownFlags))
+        return FB_ERR_INVALID_VALUE;
+    const Plan &pl = cached_plan(W, batch, sms, (flags & FB_GEMV_INDEPENDENT) != 0);
+    out[0] = pl.C;
+    out[1] = pl.cpb;
+    out[2] = pl.RB;
+    out[3] = pl.nwarps;
+    out[4] = (int)pl.smem;
+    out[5] = pl.V;
+    return FB_OK;
+}
+
 extern "C" fb_status fb_gemv(const fb_weights *W, const void *x, fb_dtype t, float *y, void *ws,
                              size_t ws_bytes, unsigned flags, void *stream) {
     if (!W) return FB_ERR_INVALID_VALUE;
     return fb_gemv_batched(W, x, t, 1, W->N, y, W->M, ws, ws_bytes, flags, stream);
+}
+
+extern "C" fb_status fb_device_errors(unsigned int *flags, int clear) {
+    if (!flags) return FB_ERR_INVALID_VALUE;
+    if (cudaDeviceSynchronize() != cudaSuccess) return FB_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(flags, g_error_flags, sizeof(unsigned int)) != cudaSuccess) return FB_ERR_CUDA;
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_flags, &zero, sizeof(unsigned int)) != cudaSuccess) return FB_ERR_CUDA;
+    }
+    return FB_OK;
 }

@@ -153,6 +153,37 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert L.fb_validate_weights(None) == INVALID
 
 
+@pytest.mark.parametrize("shape", [
+    (256, 256, 2, 4, 0, 0), (4096, 4096, 2, 4, 128, 2), (11008, 4096, 2, 4, 123, 2),
+    (4096, 11008, 2, 4, 330, 2), (8192, 8192, 3, 8, 410, 2), (28672, 8192, 3, 8, 410, 2),
+    (8192, 28672, 3, 8, 1434, 2), (131077, 64, 1, 2, 0, 0), (100, 800, 4, 1, 800, 4),
+])
+@pytest.mark.parametrize("batch", [1, 16])
+@pytest.mark.parametrize("flags", [0, 1, 3])
+def test_launch_plan_covers_the_matrix(L, shape, batch, flags):
+    M, N, K, g, nS, Ks = shape
+    s = fake_weights(M=M, N=N, K=K, g=g, nS=nS, Ks=Ks)
+    plan = fb.fb_gemv_launch_plan(s, batch, flags, 148)
+    nchunks = -(-M // 32)
+    P = lambda n: -(-n // 256)
+    V = P(N) * K + (P(-(-nS // 32) * 32) * Ks if nS else 0)
+    assert plan["V"] == V
+    assert 1 <= plan["C"] <= min(8, V)
+    assert plan["RB"] * plan["cpb"] >= nchunks > (plan["RB"] - 1) * plan["cpb"]
+    assert plan["warps"] == 8
+    assert 0 < plan["smem"] <= 200 * 1024
+
+
+def test_launch_plan_rejects_bad_arguments(L):
+    s = fake_weights()
+    out = (C.c_int * 6)()
+    assert L.fb_gemv_launch_plan(C.byref(s), 1, 4, 148, C.cast(out, C.c_void_p)) == INVALID   # unknown flag
+    assert L.fb_gemv_launch_plan(C.byref(s), 0, 0, 148, C.cast(out, C.c_void_p)) == INVALID   # batch 0
+    assert L.fb_gemv_launch_plan(C.byref(s), 1, 0, 0, C.cast(out, C.c_void_p)) == INVALID     # sms 0
+    assert L.fb_gemv_launch_plan(C.byref(s), 1, 0, 148, None) == INVALID
+    assert L.fb_device_errors(None, 0) == INVALID
+
+
 def test_layout_spec_is_a_bijection():
     """Every (base, row, column) lands on its own bit of the packed buffer."""
     rng = np.random.default_rng(0)

@@ -301,3 +301,12 @@ def test_workload_70b(shape_index, batch):
     if batch == 4:
         pi = wl.layer70b(shape_index, batch, integer_mode=True)
         check(pi, run_gpu(pi), sample_rows(pi.M, 64, 10 + shape_index))
+
+
+@pytest.mark.gpu
+def test_device_error_flags_stay_clear():
+    # every bounded wait for a weight copy in the runs above ended in time
+    p = wl.layer4096()
+    W = fb.Weights.from_problem(p)
+    fb.fb_gemv(W, torch.from_numpy(p.x[0]).cuda(), flags=fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT)
+    assert fb.fb_device_errors(clear=True) == 0
