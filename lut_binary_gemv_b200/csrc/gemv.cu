@@ -11,11 +11,11 @@
 // chunks; CTA j of the cluster takes a contiguous, balanced slice of the V
 // virtual panels, so the cluster covers every column of its rows.
 //
-// Per CTA (8 warps; warp w owns chunks w, w+8, ... of the row block):
-//   1. before the programmatic-launch wait: the first weight items of every
-//      warp start streaming into the warp's ring of shared-memory slots (one
-//      bulk asynchronous copy per item, completion on an mbarrier), and the
-//      row scales of the row block are staged in shared memory;
+// Per CTA (16 warps; warp w owns chunks w and w+16 of the row block):
+//   1. before the programmatic-launch wait: the weights of the first panels
+//      start streaming into shared-memory slots (one bulk asynchronous copy
+//      per panel of the row block, completion on an mbarrier), and the row
+//      scales and per-panel descriptors are staged in shared memory;
 //   2. per panel, all 256 threads build its byte tables in shared memory
 //      (LUT-BSF: z = alpha_c * x, salient panels reading x[s_idx[t]] -- the
 //      virtual columnar mapping -- and for each group of 8 columns the 256
@@ -45,6 +45,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <new>
+#include <type_traits>
 
 #include "fb_internal.cuh"
 
@@ -54,10 +55,9 @@ namespace fb {
 namespace {
 
 constexpr int kMaxCluster = 8;
-constexpr int kNW = 8;                  // warps per CTA
-constexpr int kMaxCpb = 16;             // chunks per row block (two per warp)
-constexpr size_t kMaxDynSmem = 200 * 1024;   // dynamic shared memory per CTA
-constexpr double kOverlapDepth = 8;          // launches in flight together, for the planner
+constexpr int kNW = 16;                 // warps per CTA
+constexpr int kMaxCpb = 32;             // chunks per row block (four per warp)
+constexpr size_t kMaxDynSmem = 225 * 1024;   // dynamic shared memory per CTA
 constexpr size_t kSmemPerSM = 228 * 1024;
 constexpr size_t kStaticSmem = 1024;          // the kernel's static shared memory, rounded up
 constexpr unsigned kKnownFlags = FB_GEMV_PDL | FB_GEMV_INDEPENDENT;
@@ -205,9 +205,8 @@ __device__ __forceinline__ void sums16(float z0, float z1, float z2, float z3, f
     for (int a = 0; a < 16; ++a) e[a] = __fadd_rn(p01[a & 3], p23[a >> 2]);
 }
 
-// One virtual panel: where its words live, its width and its scales.
+// One virtual panel: its width, its scales and its columns.
 struct VPanel {
-    const uint8_t *pl;   // chunk block 0 of this panel and base
     const float *ac;     // column scales of this base, or null (all ones)
     int col0;            // first column of the panel (global, or compact salient)
     int Bp;              // byte groups (width / 8)
@@ -231,16 +230,6 @@ __device__ __forceinline__ PanelPos panel_pos(const GemvArgs &a, int v) {
     return q;
 }
 
-__device__ __forceinline__ void panel_next(const GemvArgs &a, PanelPos &q) {
-    if (++q.p == (q.sal ? a.Ps : a.Pg)) {
-        q.p = 0;
-        if (++q.k == (q.sal ? a.Ks : a.K)) {
-            q.sal = 1;
-            q.k = 0;
-        }
-    }
-}
-
 __device__ __forceinline__ VPanel panel_at(const GemvArgs &a, const PanelPos &q) {
     const int ncols = q.sal ? a.nS_pad : a.N;
     VPanel r;
@@ -248,28 +237,53 @@ __device__ __forceinline__ VPanel panel_at(const GemvArgs &a, const PanelPos &q)
     r.kb = q.sal ? a.K + q.k : q.k;
     r.col0 = q.p * kPanelCols;
     r.Bp = panel_width(ncols, q.p) >> 3;
-    r.pl = (q.sal ? a.s_planes : a.planes) + (size_t)q.k * a.M_pad * (size_t)(ncols / 8) +
-           (size_t)32 * q.p * a.M_pad;
     r.ac = q.sal ? a.s_alpha_c + (size_t)q.k * a.nS : (a.alpha_c ? a.alpha_c + (size_t)q.k * a.N : nullptr);
     return r;
+}
+
+// Chunk block 0 of a virtual panel in its planes buffer.
+__device__ __forceinline__ const uint8_t *panel_planes(const GemvArgs &a, const PanelPos &q) {
+    const int ncols = q.sal ? a.nS_pad : a.N;
+    return (q.sal ? a.s_planes : a.planes) + (size_t)q.k * a.M_pad * (size_t)(ncols / 8) +
+           (size_t)32 * q.p * a.M_pad;
+}
+
+// What a CTA needs of one of its panels, built once per CTA in shared
+// memory: width, row-scale base, salient flag, first column, scales, words.
+struct PanelDesc {
+    const float *ac;      // column scales of the panel's base, or null (all ones)
+    const uint8_t *pl;    // chunk block 0 of the panel
+    int bp_kb_sal;        // Bp | kb << 8 | sal << 16
+    int col0;
+};
+
+__device__ __forceinline__ PanelDesc panel_desc(const GemvArgs &a, int v) {
+    const PanelPos q = panel_pos(a, v);
+    const VPanel vp = panel_at(a, q);
+    PanelDesc d;
+    d.ac = vp.ac;
+    d.pl = panel_planes(a, q);
+    d.bp_kb_sal = vp.Bp | vp.kb << 8 | vp.sal << 16;
+    d.col0 = vp.col0;
+    return d;
 }
 
 // Column c of a panel: its scale alpha_c and the column of x it reads (-1:
 // none, including the columns past a narrow panel's width, which therefore
 // build all-zero table columns).
-__device__ __forceinline__ void column_source(const GemvArgs &a, const VPanel &vp, int c, float &ac, int &xi) {
+__device__ __forceinline__ void column_source(const GemvArgs &a, const PanelDesc &d, int c, float &ac, int &xi) {
     ac = 0.0f;
     xi = -1;
-    if (c >= vp.Bp * 8) return;
-    const int col = vp.col0 + c;
-    if (!vp.sal) {
+    if (c >= (d.bp_kb_sal & 255) * 8) return;
+    const int col = d.col0 + c;
+    if (!(d.bp_kb_sal >> 16)) {
         xi = col;
-        if (vp.ac)
-            ac = __ldg(vp.ac + col);
+        if (d.ac)
+            ac = __ldg(d.ac + col);
         else
             ac = 1.0f;
     } else if (col < a.nS) {
-        ac = __ldg(vp.ac + col);
+        ac = __ldg(d.ac + col);
         const uint32_t jx = __ldg(a.s_idx + col);
         xi = jx < (uint32_t)a.N ? (int)jx : -1;   // an invalid index contributes 0
     }
@@ -332,23 +346,25 @@ __device__ __forceinline__ float lookup_row(const uint32_t (&w)[8], const uint32
 // entry b = T_lo[b & 15] + T_hi[b >> 4], where T_lo and T_hi are the 16-entry
 // tables of the group's low and high 4 columns, each (+-z0 +- z1) + (+-z2 +-
 // z3).  Columns past a narrow panel's width have z = 0, so their entries are
-// 0.  T points at the buffer (entry b of group q at T[b*64 + q]).
+// 0.  T points at the buffer (entry b of group q at T[b*64 + q]).  Each of
+// the kNW warps writes 256 / kNW consecutive entries b of every group.
 __device__ __forceinline__ void build_byte_table(const float *zp, float *T, int warp, int lane) {
+    constexpr int kHi = 16 / kNW;   // high-nibble values per warp: entries b = 16*kHi*warp ...
     const float4 za = *reinterpret_cast<const float4 *>(zp + 8 * lane);
     const float4 zb = *reinterpret_cast<const float4 *>(zp + 8 * lane + 4);
     float lo[16];
     sums16(za.x, za.y, za.z, za.w, lo);
-    float hi[2];
+    float hi[kHi];
 #pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2) {
-        const int h = 2 * warp + s2;
+    for (int s2 = 0; s2 < kHi; ++s2) {
+        const int h = kHi * warp + s2;
         const float s01 = __fadd_rn((h & 1) ? zb.x : -zb.x, (h & 2) ? zb.y : -zb.y);
         const float s23 = __fadd_rn((h & 4) ? zb.z : -zb.z, (h & 8) ? zb.w : -zb.w);
         hi[s2] = __fadd_rn(s01, s23);
     }
-    float *col = T + (32 * warp) * 64 + lane;
+    float *col = T + (16 * kHi * warp) * 64 + lane;
 #pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2)
+    for (int s2 = 0; s2 < kHi; ++s2)
 #pragma unroll
         for (int v = 0; v < 16; ++v) col[(16 * s2 + v) * 64] = __fadd_rn(lo[v], hi[s2]);
 }
@@ -386,17 +402,17 @@ __device__ __forceinline__ void read_item_full(const uint8_t *slot, int lane, ui
 }
 
 // Shared-memory layout of one CTA (bytes): two interleaved byte tables |
-// z of two panels | two weight slots | row scales [KB][R] | row partials [R]
-// | cluster inbox.
+// z of two panels | kSlots weight slots of cpb KiB | row scales [KB][R] |
+// row partials [R] | cluster inbox [R + C].
 constexpr int kTableBytes = 65536;
 constexpr int kZBytes = 2 * kPanelCols * 4;
-constexpr int kSlotBytes = kMaxCpb * 1024;   // one panel of a row block: cpb blocks of <= 1 KiB
+constexpr int kSlots = 3;
 constexpr int kItemsPerWarp = kMaxCpb / kNW;
 
 template <int XT>
-__global__ void __launch_bounds__(kNW * 32, 2) gemv_kernel(const __grid_constant__ GemvArgs args) {
+__global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant__ GemvArgs args) {
     extern __shared__ __align__(128) float smem_f[];
-    __shared__ __align__(8) unsigned long long s_bar[2];
+    __shared__ __align__(8) unsigned long long s_bar[kSlots];
     // The launch's parameter block is new to every SM's constant cache, and the
     // kernel would touch its fields one after another, each a miss; one
     // parallel copy into shared memory pays that latency once.
@@ -406,8 +422,8 @@ __global__ void __launch_bounds__(kNW * 32, 2) gemv_kernel(const __grid_constant
     for (int i = tid; i < (int)(sizeof(GemvArgs) / 4); i += blockDim.x)
         reinterpret_cast<int *>(&s_args)[i] = reinterpret_cast<const int *>(&args)[i];
     if (tid == 0) {
-        mbar_init(smem_addr(&s_bar[0]));
-        mbar_init(smem_addr(&s_bar[1]));
+#pragma unroll
+        for (int s2 = 0; s2 < kSlots; ++s2) mbar_init(smem_addr(&s_bar[s2]));
         mbar_init_fence();
     }
     __syncthreads();
@@ -422,42 +438,43 @@ __global__ void __launch_bounds__(kNW * 32, 2) gemv_kernel(const __grid_constant
     const int KB = a.K + a.Ks;                          // bases with row scales: global, then salient
     const bool independent = (a.flags & FB_GEMV_INDEPENDENT) != 0;
     const size_t xoff = (size_t)b * a.ldx;
+    const int slot_bytes = cpb * 1024;
 
     float *tables = smem_f;
     float *zbuf = smem_f + kTableBytes / 4;
     uint8_t *slots = reinterpret_cast<uint8_t *>(smem_f) + kTableBytes + kZBytes;
-    float *s_ar = smem_f + (kTableBytes + kZBytes + 2 * kSlotBytes) / 4;
+    float *s_ar = reinterpret_cast<float *>(slots + kSlots * slot_bytes);
     float *pw = s_ar + KB * R;
     float *part = pw + R;
+    PanelDesc *s_desc = reinterpret_cast<PanelDesc *>(part + ((R + kMaxCluster + 1) & ~1));
     const uint32_t slots_s = smem_addr(slots), bar_s = smem_addr(&s_bar[0]);
 
     // ---- 1. weight copies and row scales, before the wait -------------------
     // Panel vi's blocks of this row block are contiguous: one bulk copy into
-    // slot vi % 2, issued by thread 0.
+    // slot vi % kSlots, issued by thread 0 kSlots - 1 panels ahead of use.
     uint32_t pending = 0, pend_par = 0;   // thread 0: slots with a copy in flight, its phase parity
-    auto issue = [&](int vi, const VPanel &vp) {
-        const uint32_t blk = 32u * (uint32_t)vp.Bp;
-        bulk_load(slots_s + (vi & 1) * kSlotBytes, vp.pl + (size_t)blk * c_first, blk * (uint32_t)nvalid,
-                  bar_s + 8 * (vi & 1));
-        pending |= 1u << (vi & 1);
-        pend_par = (pend_par & ~(1u << (vi & 1))) | ((uint32_t)(vi >> 1) & 1u) << (vi & 1);
+    auto issue = [&](int vi, const PanelDesc &d) {
+        const int s2 = vi % kSlots;
+        const uint32_t blk = 32u * (uint32_t)(d.bp_kb_sal & 255);
+        bulk_load(slots_s + s2 * slot_bytes, d.pl + (size_t)blk * c_first, blk * (uint32_t)nvalid, bar_s + 8 * s2);
+        pending |= 1u << s2;
+        pend_par = (pend_par & ~(1u << s2)) | ((uint32_t)(vi / kSlots) & 1u) << s2;
     };
-    PanelPos pos_cur = panel_pos(a, vb), pos_ahead = pos_cur;   // panels vi and vi + 2
-    if (n_v > 0 && tid == 0) issue(0, panel_at(a, pos_ahead));
-    panel_next(a, pos_ahead);
-    if (n_v > 1 && tid == 0) issue(1, panel_at(a, pos_ahead));
-    panel_next(a, pos_ahead);
+    if (tid == 0)
+        for (int v = 0; v < kSlots - 1 && v < n_v; ++v) issue(v, panel_desc(a, vb + v));
+    for (int t = tid; t < n_v; t += blockDim.x) s_desc[t] = panel_desc(a, vb + t);
 
     // column data of one panel: thread t stages column t
     float z_ac = 0.0f;
     uint32_t z_x = 0;
     int z_xi = -1;
-    auto stage = [&](const VPanel &vp, bool read_x) {
+    auto stage = [&](const PanelDesc &d, bool read_x) {
         z_x = 0;
-        column_source(a, vp, tid, z_ac, z_xi);
+        if (tid >= kPanelCols) return;
+        column_source(a, d, tid, z_ac, z_xi);
         if (read_x && z_xi >= 0) z_x = load_x_bits<XT>(a.x, xoff + z_xi);
     };
-    if (n_v > 0) stage(panel_at(a, pos_cur), independent);
+    if (n_v > 0) stage(panel_desc(a, vb), independent);
     griddep_launch_dependents();
     // the row block's row scales, every base (rows past M: 0)
     for (int t = tid; t < KB * R; t += blockDim.x) {
@@ -471,93 +488,84 @@ __global__ void __launch_bounds__(kNW * 32, 2) gemv_kernel(const __grid_constant
         griddep_wait();
         if (z_xi >= 0) z_x = load_x_bits<XT>(a.x, xoff + z_xi);
     }
-    zbuf[tid] = z_xi >= 0 ? __fmul_rn(z_ac, x_value<XT>(z_x)) : 0.0f;
-    if (n_v > 1) {
-        PanelPos p1 = pos_cur;
-        panel_next(a, p1);
-        stage(panel_at(a, p1), true);
-    }
-    __syncthreads();   // z of panel 0 and row scales written
+    if (tid < kPanelCols) zbuf[tid] = z_xi >= 0 ? __fmul_rn(z_ac, x_value<XT>(z_x)) : 0.0f;
+    __syncthreads();   // z of panel 0, panel descriptors and row scales written
+    if (n_v > 1) stage(s_desc[1], true);
 
     // column offsets of a full panel (narrow panels compute theirs)
     uint32_t off_full[8];
     full_offsets(lane, off_full);
 
     // ---- 3. per panel: its byte tables, then this warp's chunks -------------
-    // Warp w owns chunks w and w + 8 of the row block; each lane keeps its
-    // two rows' partial sums and current row scales in registers.  The words
-    // move to registers before the panel's barrier, so right after it the
-    // slot can take the panel two ahead.
+    // Warp w owns chunks w + kNW * i of the row block; each lane keeps its
+    // rows' partial sums and current row scales in registers.  The barrier of
+    // panel vi also ends every warp's reads of panel vi - 1, whose slot then
+    // takes panel vi + kSlots - 1.
     bool failed = false;
     float racc[kItemsPerWarp], rar[kItemsPerWarp];
 #pragma unroll
     for (int it = 0; it < kItemsPerWarp; ++it) racc[it] = rar[it] = 0.0f;
-    int kb_cur = -1;
-#pragma unroll 1
-    for (int vi = 0; vi < n_v; ++vi) {
-        const int buf = vi & 1;
-        const VPanel vp = panel_at(a, pos_cur);
-        const int Bp = vp.Bp;
-        uint32_t w[kItemsPerWarp][8];
+    int kb_cur = -1, sl = 0;   // sl = vi % kSlots
+    // One panel; the table buffer is a compile-time constant in each of the
+    // two copies, so table addresses fold into the shared loads.
+    auto panel = [&](auto bufc, int vi) {
+        constexpr int buf = decltype(bufc)::value;
+        const int bks = s_desc[vi].bp_kb_sal;
+        const int Bp = bks & 255, kb = (bks >> 8) & 255;
         bool ok = !failed;
         if (ok) {
-            const uint32_t par = (uint32_t)(vi >> 1) & 1u;
-            ok = mbar_try_wait(bar_s + 8 * buf, par) || mbar_wait_bounded(bar_s + 8 * buf, par);
+            const uint32_t par = (uint32_t)(vi / kSlots) & 1u;
+            ok = mbar_try_wait(bar_s + 8 * sl, par) || mbar_wait_bounded(bar_s + 8 * sl, par);
         }
-        if (tid == 0 && ok) pending &= ~(1u << buf);
-        const uint8_t *slot = slots + buf * kSlotBytes;
-#pragma unroll
-        for (int it = 0; it < kItemsPerWarp; ++it) {
-            const int cl = warp + kNW * it;
-#pragma unroll
-            for (int m = 0; m < 8; ++m) w[it][m] = 0;
-            if (ok && cl < nvalid) {
-                if (Bp == 32) {
-                    read_item_full(slot + cl * 1024, lane, w[it]);
-                } else {
-                    const Words r = read_item_narrow(slot + cl * 32 * Bp, Bp, lane);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) w[it][m] = r.w[m];
-                }
-            }
-        }
+        if (tid == 0 && ok) pending &= ~(1u << sl);
         float *tb = tables + 32 * buf;
         build_byte_table(zbuf + buf * kPanelCols, tb, warp, lane);
-        if (vi + 1 < n_v) {   // z of the next panel into the other buffer
+        if (vi + 1 < n_v && tid < kPanelCols)   // z of the next panel into the other buffer
             zbuf[(buf ^ 1) * kPanelCols + tid] = z_xi >= 0 ? __fmul_rn(z_ac, x_value<XT>(z_x)) : 0.0f;
-        }
-        VPanel vp2;
-        if (vi + 2 < n_v) {
-            vp2 = panel_at(a, pos_ahead);
-            stage(vp2, true);
-        }
-        panel_next(a, pos_cur);
-        panel_next(a, pos_ahead);
-        // tables of panel vi complete, the slot read, the other table's readers done
+        if (vi + 2 < n_v) stage(s_desc[vi + 2], true);
+        // tables of panel vi complete; every warp done with panel vi - 1
         failed = __syncthreads_or(!ok) != 0;
-        if (failed) continue;
-        if (tid == 0 && vi + 2 < n_v) issue(vi + 2, vp2);
-        if (vp.kb != kb_cur) {   // a new base: its row scales
-            kb_cur = vp.kb;
+        if (failed) return;
+        if (tid == 0 && vi + kSlots - 1 < n_v) issue(vi + kSlots - 1, s_desc[vi + kSlots - 1]);
+        if (kb != kb_cur) {   // a new base: its row scales
+            kb_cur = kb;
 #pragma unroll
             for (int it = 0; it < kItemsPerWarp; ++it) {
                 const int cl = warp + kNW * it;
                 if (cl < cpb) rar[it] = s_ar[kb_cur * R + cl * kChunkRows + lane];
             }
         }
-        uint32_t offp[8];
+        const uint8_t *slot = slots + sl * slot_bytes;
+        sl = sl + 1 == kSlots ? 0 : sl + 1;
         if (Bp == 32) {
 #pragma unroll
-            for (int m = 0; m < 8; ++m) offp[m] = off_full[m];
+            for (int it = 0; it < kItemsPerWarp; ++it) {
+                const int cl = warp + kNW * it;
+                if (cl < nvalid) {
+                    uint32_t w[8];
+                    read_item_full(slot + cl * 1024, lane, w);
+                    racc[it] = __fadd_rn(racc[it], __fmul_rn(rar[it], lookup_row(w, off_full, tb)));
+                }
+            }
         } else {
             const Offsets o = narrow_offsets(lane, Bp);
+#pragma unroll 1
+            for (int it = 0; it < kItemsPerWarp; ++it) {
+                const int cl = warp + kNW * it;
+                if (cl < nvalid) {
+                    const Words r = read_item_narrow(slot + cl * 32 * Bp, Bp, lane);
+                    const float sum = lookup_row(r.w, o.w, tb);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) offp[m] = o.w[m];
+                    for (int i2 = 0; i2 < kItemsPerWarp; ++i2)
+                        if (i2 == it) racc[i2] = __fadd_rn(racc[i2], __fmul_rn(rar[i2], sum));
+                }
+            }
         }
-#pragma unroll
-        for (int it = 0; it < kItemsPerWarp; ++it) {
-            if (warp + kNW * it < nvalid) racc[it] = __fadd_rn(racc[it], __fmul_rn(rar[it], lookup_row(w[it], offp, tb)));
-        }
+    };
+#pragma unroll 1
+    for (int vi = 0; vi < n_v; vi += 2) {
+        panel(std::integral_constant<int, 0>{}, vi);
+        if (vi + 1 < n_v) panel(std::integral_constant<int, 1>{}, vi + 1);
     }
 #pragma unroll
     for (int it = 0; it < kItemsPerWarp; ++it) {
@@ -567,7 +575,7 @@ __global__ void __launch_bounds__(kNW * 32, 2) gemv_kernel(const __grid_constant
     if (failed && tid == 0) {
         // Wait (bounded) for the copies still in flight, so none lands after
         // the CTA has gone, then flag the failure.
-        for (int s2 = 0; s2 < 2; ++s2)
+        for (int s2 = 0; s2 < kSlots; ++s2)
             if (pending & (1u << s2)) mbar_wait_bounded(bar_s + 8 * s2, (pend_par >> s2) & 1u);
         atomicOr(&g_error_flags, 1u);
     }
@@ -645,18 +653,21 @@ void split_panels(int V, int C, int *vsplit, int *max_n) {
 // Dynamic shared memory of a CTA with cpb chunks of rows and KB bases:
 // tables, z, rings, row scales, row partials and the inbox of row partials
 // pushed by the cluster (C * ceil(R / C) <= R + C floats).
-size_t smem_for(int cpb, int KB) {
+size_t smem_for(int cpb, int KB, int nv) {
     const size_t R = (size_t)cpb * kChunkRows;
-    return (size_t)kTableBytes + kZBytes + 2 * (size_t)kSlotBytes + R * KB * 4 + R * 4 + (R + kMaxCluster) * 4;
+    return (size_t)kTableBytes + kZBytes + (size_t)kSlots * cpb * 1024 + R * KB * 4 + R * 4 +
+           ((R + kMaxCluster + 1) & ~(size_t)1) * 4 + (size_t)nv * sizeof(PanelDesc);
 }
 
 // The launch plan: cluster size C (the split of the V virtual panels over
-// the cluster's CTAs) and row block size (cpb chunks of 32 rows).  Chosen
-// by a cost model in SM cycles.  Per panel a CTA writes 32 KiB of tables
-// (256 shared-memory store cycles) and, per chunk of its rows, reads 1 KiB
-// of weights through the shared-memory pipe and makes 32 table lookups
-// (48 cycles); latencies: a panel's build and barrier, an item per warp, a
-// fixed prologue and reduction.
+// the cluster's CTAs) and row block size (cpb chunks of 32 rows).
+//  * Calls flagged independent overlap their neighbours, so the plan that
+//    does the least work wins: the largest row blocks (fewest table builds
+//    per row), C = 2 for matrices of few row blocks, else 1.
+//  * A dependent call is timed alone: its latency is about a fixed 4 us plus
+//    1.2 us per panel a CTA works through (build, barrier, lookups), times
+//    the number of waves; more CTAs per cluster shorten a CTA's panel list.
+// Both rules were fitted to timings of this kernel on B200.
 Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
     Plan pl;
     pl.M_pad = round_up(W->M, kChunkRows);
@@ -667,43 +678,46 @@ Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
     pl.nchunks = pl.M_pad / kChunkRows;
     pl.nwarps = kNW;
     const int KB = W->K + (W->nS > 0 ? W->Ks : 0);
-    const double build_mio = 256, item_mio = 48;          // shared-memory pipe cycles
-    const double build_lat = 500, item_lat = 700, fixed = 4000;   // latency, cycles
-    double best = 1e300;
-    pl.C = 1;
-    pl.cpb = 1;
-    pl.RB = pl.nchunks;
-    pl.vsplit[0] = 0;
-    pl.vsplit[1] = pl.V;
-    for (int C = 1; C <= std::min(kMaxCluster, pl.V); ++C) {
+    const int occ_regs = 65536 / (kNW * 32 * 128);   // CTAs per SM by registers (128 per thread)
+    auto fits = [&](int C, int cpb) {
         int vs[kMaxCluster + 1], nvm;
         split_panels(pl.V, C, vs, &nvm);
-        for (int cpb = 1; cpb <= std::min(kMaxCpb, pl.nchunks); ++cpb) {
-            const int RB = ceil_div(pl.nchunks, cpb);
-            if (RB > 65535) continue;
-            if (cpb > 1 && ceil_div(pl.nchunks, cpb - 1) == RB) continue;   // same split, fewer rows
-            const size_t smem = smem_for(cpb, KB);
-            if (smem > kMaxDynSmem) continue;
-            const int occ = smem + kStaticSmem + 1024 <= kSmemPerSM / 2 ? 2 : 1;
-            const long ctas = (long)C * RB * batch;
-            const double mio = nvm * (build_mio + item_mio * cpb);   // per CTA
-            const double lat = fixed + nvm * (build_lat + std::ceil((double)cpb / kNW) * item_lat);
-            const double waves = std::ceil((double)ctas / ((double)sms * occ));
-            const double per_sm = std::ceil((double)ctas / sms) * mio;
-            // A dependent call is timed alone: its critical path counts.  Calls
-            // flagged independent overlap their neighbours, so what counts is
-            // the SM time they occupy, plus a share of one CTA's latency for
-            // the launches that do not overlap.
-            const double cost =
-                independent ? std::max((double)ctas * lat / ((double)sms * occ), (double)ctas * mio / sms) +
-                                  lat / kOverlapDepth
-                            : std::max(per_sm, waves * lat);
-            if (cost < best * 0.999) {
-                best = cost;
-                pl.C = C;
-                pl.cpb = cpb;
-                pl.RB = RB;
-                std::copy(vs, vs + C + 1, pl.vsplit);
+        return smem_for(cpb, KB, nvm) <= kMaxDynSmem;
+    };
+    auto set = [&](int C, int cpb) {
+        pl.C = C;
+        pl.RB = ceil_div(pl.nchunks, cpb);
+        pl.cpb = ceil_div(pl.nchunks, pl.RB);   // balanced: the same rows, less padding
+        int nvm;
+        split_panels(pl.V, C, pl.vsplit, &nvm);
+    };
+    if (independent) {
+        int cpb = std::min(kMaxCpb, pl.nchunks);
+        while (cpb > 1 && !fits(2, cpb)) --cpb;
+        const int RB = ceil_div(pl.nchunks, cpb);
+        set(std::min(pl.V, RB <= 6 ? 2 : 1), cpb);
+    } else {
+        const double fixed = 4.0, per_panel = 1.2, per_item = 0.1;   // microseconds
+        double best = 1e300;
+        set(1, std::min(kMaxCpb, pl.nchunks));
+        for (int C = 1; C <= std::min(kMaxCluster, pl.V); ++C) {
+            int vs[kMaxCluster + 1], nvm;
+            split_panels(pl.V, C, vs, &nvm);
+            // at least one chunk per warp (fewer measured slower on B200)
+            for (int cpb = std::min(kNW, pl.nchunks); cpb <= std::min(kMaxCpb, pl.nchunks); ++cpb) {
+                const int RB = ceil_div(pl.nchunks, cpb);
+                if (RB > 65535) continue;
+                if (cpb > 1 && ceil_div(pl.nchunks, cpb - 1) == RB) continue;   // same split, fewer rows
+                const size_t smem = smem_for(cpb, KB, nvm);
+                if (smem > kMaxDynSmem) continue;
+                const int occ = std::max(1, std::min(occ_regs, (int)(kSmemPerSM / (smem + kStaticSmem + 1024))));
+                const long ctas = (long)C * RB * batch;
+                const double waves = std::ceil((double)ctas / ((double)sms * occ));
+                const double cost = waves * (fixed + nvm * (per_panel + std::ceil((double)cpb / kNW) * per_item));
+                if (cost < best * 0.999) {
+                    best = cost;
+                    set(C, cpb);
+                }
             }
         }
     }
@@ -714,13 +728,15 @@ Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
         if (sscanf(ov, "%d,%d", &oc, &ocpb) == 2 && oc >= 1 && ocpb >= 1) {
             pl.C = std::min(std::min(oc, kMaxCluster), pl.V);
             pl.cpb = std::min(std::min(ocpb, kMaxCpb), pl.nchunks);
-            while (pl.cpb > 1 && smem_for(pl.cpb, KB) > kMaxDynSmem) --pl.cpb;
-            pl.RB = ceil_div(pl.nchunks, pl.cpb);
             int nvm;
             split_panels(pl.V, pl.C, pl.vsplit, &nvm);
+            while (pl.cpb > 1 && smem_for(pl.cpb, KB, nvm) > kMaxDynSmem) --pl.cpb;
+            pl.RB = ceil_div(pl.nchunks, pl.cpb);
         }
     }
-    pl.smem = smem_for(pl.cpb, KB);
+    int nv_max = 0;
+    for (int jj = 0; jj < pl.C; ++jj) nv_max = std::max(nv_max, pl.vsplit[jj + 1] - pl.vsplit[jj]);
+    pl.smem = smem_for(pl.cpb, KB, nv_max);
     return pl;
 }
 

@@ -170,8 +170,8 @@ def test_launch_plan_covers_the_matrix(L, shape, batch, flags):
     assert plan["V"] == V
     assert 1 <= plan["C"] <= min(8, V)
     assert plan["RB"] * plan["cpb"] >= nchunks > (plan["RB"] - 1) * plan["cpb"]
-    assert plan["warps"] == 8
-    assert 0 < plan["smem"] <= 200 * 1024
+    assert plan["warps"] in (8, 16)
+    assert 0 < plan["smem"] <= 225 * 1024
 
 
 def test_launch_plan_rejects_bad_arguments(L):
