@@ -341,6 +341,30 @@ __device__ __forceinline__ float lookup_row(const uint32_t (&w)[8], const uint32
     return __fadd_rn(__fadd_rn(f2sum(acc[0]), f2sum(acc[1])), __fadd_rn(f2sum(acc[2]), f2sum(acc[3])));
 }
 
+// Two rows' lookups interleaved (twice the independent shared loads in
+// flight); each sum is accumulated in the same order as lookup_row's.
+__device__ __forceinline__ void lookup_rows2(const uint32_t (&wa)[8], const uint32_t (&wb)[8],
+                                             const uint32_t (&offp)[8], const float *tbl, float &sa, float &sb) {
+    unsigned long long acc_a[4] = {0, 0, 0, 0}, acc_b[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const float a0 = lds(tbl, prmt(wa[m], offp[m], addr_sel(0)));
+        const float b0 = lds(tbl, prmt(wb[m], offp[m], addr_sel(0)));
+        const float a1 = lds(tbl, prmt(wa[m], offp[m], addr_sel(1)));
+        const float b1 = lds(tbl, prmt(wb[m], offp[m], addr_sel(1)));
+        const float a2 = lds(tbl, prmt(wa[m], offp[m], addr_sel(2)));
+        const float b2 = lds(tbl, prmt(wb[m], offp[m], addr_sel(2)));
+        const float a3 = lds(tbl, prmt(wa[m], offp[m], addr_sel(3)));
+        const float b3 = lds(tbl, prmt(wb[m], offp[m], addr_sel(3)));
+        acc_a[(2 * m) & 3] = fadd2(acc_a[(2 * m) & 3], f2pack(a0, a1));
+        acc_b[(2 * m) & 3] = fadd2(acc_b[(2 * m) & 3], f2pack(b0, b1));
+        acc_a[(2 * m + 1) & 3] = fadd2(acc_a[(2 * m + 1) & 3], f2pack(a2, a3));
+        acc_b[(2 * m + 1) & 3] = fadd2(acc_b[(2 * m + 1) & 3], f2pack(b2, b3));
+    }
+    sa = __fadd_rn(__fadd_rn(f2sum(acc_a[0]), f2sum(acc_a[1])), __fadd_rn(f2sum(acc_a[2]), f2sum(acc_a[3])));
+    sb = __fadd_rn(__fadd_rn(f2sum(acc_b[0]), f2sum(acc_b[1])), __fadd_rn(f2sum(acc_b[2]), f2sum(acc_b[3])));
+}
+
 // LUT-BSF for one virtual panel, built by the whole CTA: lane q builds byte
 // group q (columns 8q .. 8q+7, z in zp), warp w its entries b = 32w .. 32w+31:
 // entry b = T_lo[b & 15] + T_hi[b >> 4], where T_lo and T_hi are the 16-entry
@@ -465,16 +489,23 @@ __global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant
     for (int t = tid; t < n_v; t += blockDim.x) s_desc[t] = panel_desc(a, vb + t);
 
     // column data of one panel: thread t stages column t
-    float z_ac = 0.0f;
-    uint32_t z_x = 0;
-    int z_xi = -1;
-    auto stage = [&](const PanelDesc &d, bool read_x) {
-        z_x = 0;
-        if (tid >= kPanelCols) return;
-        column_source(a, d, tid, z_ac, z_xi);
-        if (read_x && z_xi >= 0) z_x = load_x_bits<XT>(a.x, xoff + z_xi);
+    // Two register sets, for panels of even and odd index: panel p is staged
+    // two panels before its z is written (the loop below is unrolled by two,
+    // so the set is chosen at compile time).
+    struct Staged {
+        float ac;
+        uint32_t x;
+        int xi;
     };
-    if (n_v > 0) stage(panel_desc(a, vb), independent);
+    Staged st[2] = {{0.0f, 0u, -1}, {0.0f, 0u, -1}};
+    auto stage = [&](Staged &t, const PanelDesc &d, bool read_x) {
+        t.x = 0;
+        if (tid >= kPanelCols) return;
+        column_source(a, d, tid, t.ac, t.xi);
+        if (read_x && t.xi >= 0) t.x = load_x_bits<XT>(a.x, xoff + t.xi);
+    };
+    auto z_of = [&](const Staged &t) { return t.xi >= 0 ? __fmul_rn(t.ac, x_value<XT>(t.x)) : 0.0f; };
+    if (n_v > 0) stage(st[0], panel_desc(a, vb), independent);
     griddep_launch_dependents();
     // the row block's row scales, every base (rows past M: 0)
     for (int t = tid; t < KB * R; t += blockDim.x) {
@@ -486,11 +517,12 @@ __global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant
     // ---- 2. activations (may be the previous kernel's output) --------------
     if (!independent) {
         griddep_wait();
-        if (z_xi >= 0) z_x = load_x_bits<XT>(a.x, xoff + z_xi);
+        if (st[0].xi >= 0) st[0].x = load_x_bits<XT>(a.x, xoff + st[0].xi);
     }
-    if (tid < kPanelCols) zbuf[tid] = z_xi >= 0 ? __fmul_rn(z_ac, x_value<XT>(z_x)) : 0.0f;
+    if (tid < kPanelCols) zbuf[tid] = z_of(st[0]);
     __syncthreads();   // z of panel 0, panel descriptors and row scales written
-    if (n_v > 1) stage(s_desc[1], true);
+    if (n_v > 1) stage(st[1], s_desc[1], true);
+    if (n_v > 2) stage(st[0], s_desc[2], true);
 
     // column offsets of a full panel (narrow panels compute theirs)
     uint32_t off_full[8];
@@ -521,8 +553,8 @@ __global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant
         float *tb = tables + 32 * buf;
         build_byte_table(zbuf + buf * kPanelCols, tb, warp, lane);
         if (vi + 1 < n_v && tid < kPanelCols)   // z of the next panel into the other buffer
-            zbuf[(buf ^ 1) * kPanelCols + tid] = z_xi >= 0 ? __fmul_rn(z_ac, x_value<XT>(z_x)) : 0.0f;
-        if (vi + 2 < n_v) stage(s_desc[vi + 2], true);
+            zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
+        if (vi + 3 < n_v) stage(st[buf ^ 1], s_desc[vi + 3], true);
         // tables of panel vi complete; every warp done with panel vi - 1
         failed = __syncthreads_or(!ok) != 0;
         if (failed) return;
@@ -537,15 +569,20 @@ __global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant
         }
         const uint8_t *slot = slots + sl * slot_bytes;
         sl = sl + 1 == kSlots ? 0 : sl + 1;
-        if (Bp == 32) {
-#pragma unroll
-            for (int it = 0; it < kItemsPerWarp; ++it) {
-                const int cl = warp + kNW * it;
-                if (cl < nvalid) {
-                    uint32_t w[8];
-                    read_item_full(slot + cl * 1024, lane, w);
-                    racc[it] = __fadd_rn(racc[it], __fmul_rn(rar[it], lookup_row(w, off_full, tb)));
-                }
+        static_assert(kItemsPerWarp == 2, "the full-panel path looks up a warp's two items together");
+        if (Bp == 32 && warp + kNW < nvalid) {   // both items: interleaved
+            uint32_t w0[8], w1[8];
+            read_item_full(slot + warp * 1024, lane, w0);
+            read_item_full(slot + (warp + kNW) * 1024, lane, w1);
+            float s0, s1;
+            lookup_rows2(w0, w1, off_full, tb, s0, s1);
+            racc[0] = __fadd_rn(racc[0], __fmul_rn(rar[0], s0));
+            racc[1] = __fadd_rn(racc[1], __fmul_rn(rar[1], s1));
+        } else if (Bp == 32) {
+            if (warp < nvalid) {
+                uint32_t w[8];
+                read_item_full(slot + warp * 1024, lane, w);
+                racc[0] = __fadd_rn(racc[0], __fmul_rn(rar[0], lookup_row(w, off_full, tb)));
             }
         } else {
             const Offsets o = narrow_offsets(lane, Bp);

@@ -268,6 +268,8 @@ def test_workload_layer4096(integer_mode):
     y = run_gpu(p)
     check(p, y)
     check(p, run_gpu(p, g=8))
+    # the launch the bench times: PDL + independent (its own plan)
+    check(p, run_gpu(p, flags=fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT))
 
 
 @pytest.mark.parametrize("integer_mode", [False, True])
@@ -275,6 +277,7 @@ def test_workload_ternary(integer_mode):
     p = wl.ternary11008(integer_mode)
     y = run_gpu(p)
     check(p, y)
+    check(p, run_gpu(p, flags=fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT))
     if integer_mode:    # against the dense ternary matvec itself
         xi = p.x_f32()[0].astype(np.int64)
         want = 2.0 * p.alpha_r[0].astype(np.float64) * (p.ternary.astype(np.int64) @ xi)
@@ -282,9 +285,11 @@ def test_workload_ternary(integer_mode):
 
 
 def test_workload_7b_step():
+    indep = fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT
     for m in range(len(wl.STEP7B_MATRICES)):
         p = wl.step7b_matrix(0, m)
         check(p, run_gpu(p))
+        check(p, run_gpu(p, flags=indep))
     for layer in (13, 31):
         for m in range(len(wl.STEP7B_MATRICES)):
             p = wl.step7b_matrix(layer, m)
