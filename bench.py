@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-7b", action="store_true", help="skip the 7B-shaped step measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload timings")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile", action="store_true",
                     help="small case for ncu: 32 weight sets (142 MB), one pass per step, headline graph only")
@@ -380,6 +381,7 @@ def run_ours(args):
     step7b = None
     if not args.no_7b:
         step7b = bench_7b(args, device, stream, world, peak)
+    configs = None if args.no_configs else bench_configs(args, device, stream, world, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -400,6 +402,7 @@ def run_ours(args):
         "dependent_chain": dependent,
         "variants": {"g8_pair_tables": g8},
         "step_7b": step7b,
+        "configs": configs,
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 4),
                 "note": f"{n_e2e} eager fb_gemv calls per step from Python, pinned host x in and y out"},
@@ -446,6 +449,67 @@ def bench_7b(args, device, stream, world, peak):
             "frac_dependent_chain": round(total / (per_dep * 1e-3) / 1e9 / peak, 4),
             "algorithmic_bytes": total, "gemvs": len(Ws), "steps": steps,
             "note": "224 GEMVs, fresh x per GEMV (independent); dependent chain: each waits for its predecessor"}
+
+
+def bench_configs(args, device, stream, world, peak):
+    """Every workload of the build at its own shape: µs per call and the
+    fraction of the HBM roofline (algorithmic bytes per call, all tokens'
+    x and y included).  Distinct weight sets are rotated so that each config
+    streams more than the 126 MB L2 (except the 256x256 case, which fits in
+    L2 whatever is done).  Calls are launched as in the headline: a CUDA
+    graph of independent calls (PDL + FB_GEMV_INDEPENDENT)."""
+    import torch
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    indep = fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT
+    l2 = 126e6
+    out = {}
+
+    def measure(name, make, batches=(1,)):
+        p0 = make(0)
+        per_set = p0.algorithmic_bytes() - p0.batch * (p0.N * {"f32": 4, "f16": 2, "bf16": 2}[p0.x_dtype] + 4 * p0.M)
+        nsets = max(1, min(16, int(2 * l2 // per_set) + 1)) if per_set * 2 < 16 * l2 else 1
+        ps = [p0] + [make(i) for i in range(1, nsets)]
+        Ws = [fb.Weights.from_problem(p, device=device) for p in ps]
+        Xs = [torch.from_numpy(p.x.view(np.int16)).to(device).view(torch.bfloat16) if p.x_dtype == "bf16"
+              else torch.from_numpy(p.x).to(device) for p in ps]
+        del ps
+        res = {}
+        for B in batches:
+            Ys = [torch.empty((B, p0.M), dtype=torch.float32, device=device) for _ in Ws]
+            reps = max(-(-32 // len(Ws)), int(4 * l2 // (per_set * len(Ws))))   # >= 32 calls per graph
+
+            def body():
+                for _ in range(reps):
+                    for W, X, Y in zip(Ws, Xs, Ys):
+                        if B == 1:
+                            fb.fb_gemv(W, X[0], y=Y[0], flags=indep)
+                        else:
+                            fb.fb_gemv_batched(W, X[:B], Y=Y, flags=indep)
+            g = capture(stream, body)
+            n = max(5, args.steps // 20)
+            ms, _ = time_graph(g, stream, n, args.warmup, world)
+            calls = n * reps * len(Ws)
+            us = ms * 1e3 / calls
+            xb = {"f32": 4, "f16": 2, "bf16": 2}[p0.x_dtype]
+            nbytes = per_set + B * (p0.N * xb + 4 * p0.M)
+            gbs = nbytes / (us * 1e-6) / 1e9
+            res[f"batch{B}"] = {"us_per_call": round(us, 3), "us_per_token": round(us / B, 3), "gbs": round(gbs, 1),
+                                "frac": round(gbs / peak, 4), "weight_sets": len(Ws), "fits_l2": per_set * len(Ws) < l2}
+            del g, Ys
+        out[name] = res if len(batches) > 1 else res["batch1"]
+        del Ws, Xs
+        torch.cuda.synchronize()
+
+    measure("tiny_256x256_k2_g4", lambda i: wl.make_problem(256, 256, 2, g=4, nS=0, x_dtype="f32", alpha_dist="unit",
+                                                             seed=(5, i)))
+    measure("ternary_11008x4096", lambda i: wl.ternary11008() if i == 0 else
+            wl.make_problem(11008, 4096, 2, g=4, nS=0, x_dtype="bf16", seed=(6, i), ternary=True))
+    for si, (M, N) in enumerate(wl.SHAPES70B):
+        measure(f"layer70b_{M}x{N}_k3_g8", lambda i, si=si: wl.layer70b(si, 16) if i == 0 else
+                wl.make_problem(M, N, 3, g=8, nS=wl.salient_count(0.05, N), Ks=2, batch=16, x_dtype="f16",
+                                alpha_dist="small", seed=(7, si, i)), batches=wl.BATCHES70B)
+    return out
 
 
 def main():

@@ -700,7 +700,7 @@ size_t smem_for(int cpb, int KB, int nv) {
 // the cluster's CTAs) and row block size (cpb chunks of 32 rows).
 //  * Calls flagged independent overlap their neighbours, so the plan that
 //    does the least work wins: the largest row blocks (fewest table builds
-//    per row), C = 2 for matrices of few row blocks, else 1.
+//    per row), C = 2 for matrices of at most 8 row blocks, else 1.
 //  * A dependent call is timed alone: its latency is about a fixed 4 us plus
 //    1.2 us per panel a CTA works through (build, barrier, lookups), times
 //    the number of waves; more CTAs per cluster shorten a CTA's panel list.
@@ -732,7 +732,7 @@ Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
         int cpb = std::min(kMaxCpb, pl.nchunks);
         while (cpb > 1 && !fits(2, cpb)) --cpb;
         const int RB = ceil_div(pl.nchunks, cpb);
-        set(std::min(pl.V, RB <= 6 ? 2 : 1), cpb);
+        set(std::min(pl.V, RB <= 8 ? 2 : 1), cpb);
     } else {
         const double fixed = 4.0, per_panel = 1.2, per_item = 0.1;   // microseconds
         double best = 1e300;
