@@ -445,11 +445,38 @@ def bench_7b(args, device, stream, world, peak):
     per = run(fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT, steps)
     per_dep = run(fb.FB_GEMV_PDL, steps)
     gbs = total / (per * 1e-3) / 1e9
+
+    # Grouped: per layer q,k,v in one launch, o, gate,up in one launch, down
+    # (4 launches; x shared within a group, as in a decoder layer).
+    nm = len(wl.STEP7B_MATRICES)
+    groups = []
+    for layer in range(wl.STEP7B_LAYERS):
+        base = layer * nm
+        for ms in ((0, 1, 2), (3,), (4, 5), (6,)):
+            groups.append(([Ws[base + m] for m in ms], xs[base + ms[0]], [ys[base + m] for m in ms]))
+    xb = 2   # fp16 x
+    total_g = total - sum((len(Wg) - 1) * Wg[0].N * xb for Wg, _, _ in groups)
+
+    def run_grouped(flags, steps):
+        def body():
+            for Wg, x, yg in groups:
+                fb.fb_gemv_grouped(Wg, x, yg, flags=flags)
+        graph = capture(stream, body)
+        ms, _ = time_graph(graph, stream, steps, args.warmup, world)
+        return ms / steps
+
+    per_g = run_grouped(fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT, steps)
+    per_g_dep = run_grouped(fb.FB_GEMV_PDL, steps)
     return {"ms": round(per, 5), "gbs": round(gbs, 2), "frac": round(gbs / peak, 4),
             "ms_dependent_chain": round(per_dep, 5),
             "frac_dependent_chain": round(total / (per_dep * 1e-3) / 1e9 / peak, 4),
             "algorithmic_bytes": total, "gemvs": len(Ws), "steps": steps,
-            "note": "224 GEMVs, fresh x per GEMV (independent); dependent chain: each waits for its predecessor"}
+            "note": "224 GEMVs, fresh x per GEMV (independent); dependent chain: each waits for its predecessor",
+            "grouped": {"ms": round(per_g, 5), "frac": round(total_g / (per_g * 1e-3) / 1e9 / peak, 4),
+                        "ms_dependent_chain": round(per_g_dep, 5),
+                        "frac_dependent_chain": round(total_g / (per_g_dep * 1e-3) / 1e9 / peak, 4),
+                        "launches": len(groups), "algorithmic_bytes": total_g,
+                        "note": "fb_gemv_grouped: q,k,v and gate,up each one launch reading one x"}}
 
 
 def bench_configs(args, device, stream, world, peak):

@@ -188,6 +188,19 @@ FB_API fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtype t,
                           float *Y, int ldy, void *ws, size_t ws_bytes, unsigned flags,
                           void *stream);
 
+/* fb_gemv_grouped: one launch for n (1 <= n <= 4) weight matrices that read
+ * the same x -- the q, k, v projections of a decoder layer, or gate and up
+ * -- y[m][i] = sum_j W_hat_m[i][j] * x[j] for i < W[m]->M.  The matrices must
+ * share one format: N, K, g, nS and Ks (their data, M and salient columns
+ * are their own); otherwise FB_ERR_INVALID_VALUE.  W: n host pointers to
+ * fb_weights; y: n device pointers, y[m] holding W[m]->M floats (4-byte
+ * aligned, not aliasing x or one another).  x and flags as for fb_gemv.  The
+ * result of each matrix is the one fb_gemv gives for it with the same plan:
+ * deterministic, within the same tolerance.  FB_ERR_UNSUPPORTED if the
+ * matrices together need more than 65535 row blocks. */
+FB_API fb_status fb_gemv_grouped(const fb_weights *const *W, int n, const void *x, fb_dtype t, float *const *y,
+                                 unsigned flags, void *stream);
+
 /* fb_gemv_launch_plan: diagnostic, host only.  The launch shape fb_gemv /
  * fb_gemv_batched use for W at this batch size and these flags (calls flagged
  * FB_GEMV_INDEPENDENT get a throughput plan, others a latency plan) on a GPU

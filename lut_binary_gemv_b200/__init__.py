@@ -24,7 +24,7 @@ __all__ = [
     "FbError", "Weights", "lib", "library_path", "FB_GEMV_PDL", "FB_GEMV_INDEPENDENT",
     "fb_packed_words", "fb_pack", "fb_pack_bits", "fb_unpack", "fb_vcm_gather",
     "fb_lut_build", "fb_validate_weights", "fb_gemv_workspace_bytes", "fb_gemv",
-    "fb_gemv_batched", "fb_status_string", "fb_gemv_launch_plan", "fb_device_errors",
+    "fb_gemv_batched", "fb_status_string", "fb_gemv_launch_plan", "fb_gemv_grouped", "fb_device_errors",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -80,6 +80,7 @@ def lib() -> C.CDLL:
             "fb_gemv": (I, [W, P, I, P, P, S, C.c_uint, P]),
             "fb_gemv_batched": (I, [W, P, I, I, I, P, I, P, S, C.c_uint, P]),
             "fb_gemv_launch_plan": (I, [W, I, C.c_uint, I, P]),
+            "fb_gemv_grouped": (I, [P, I, P, I, P, C.c_uint, P]),
             "fb_device_errors": (I, [P, I]),
             "fb_status_string": (C.c_char_p, [I]),
             "fb_abi_version": (I, []),
@@ -289,3 +290,17 @@ def fb_device_errors(clear: bool = True) -> int:
     flags = C.c_uint(0)
     _check(lib().fb_device_errors(C.cast(C.byref(flags), C.c_void_p), int(clear)), "fb_device_errors")
     return flags.value
+
+
+def fb_gemv_grouped(Ws, x: torch.Tensor, ys=None, flags: int = 0):
+    """One launch for up to 4 matrices of one format that read the same x
+    (q/k/v, gate/up): returns [y_m] with y_m = W_hat_m x."""
+    n = len(Ws)
+    if ys is None:
+        ys = [torch.empty(W.M, dtype=torch.float32, device=x.device) for W in Ws]
+    wp = (C.POINTER(FbWeightsStruct) * n)(*[C.pointer(W.struct) for W in Ws])
+    yp = (C.c_void_p * n)(*[y.data_ptr() for y in ys])
+    _check(lib().fb_gemv_grouped(C.cast(wp, C.c_void_p), n, x.data_ptr(), _DTYPES[x.dtype],
+                                 C.cast(yp, C.c_void_p), flags, _stream(x.device)), "fb_gemv_grouped")
+    return ys
+

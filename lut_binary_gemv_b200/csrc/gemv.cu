@@ -42,6 +42,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <cstdio>
 #include <cstdlib>
 #include <new>
@@ -55,6 +56,7 @@ namespace fb {
 namespace {
 
 constexpr int kMaxCluster = 8;
+constexpr int kMaxGroup = 4;            // matrices in one grouped call
 constexpr int kNW = 16;                 // warps per CTA
 constexpr int kMaxCpb = 32;             // chunks per row block (four per warp)
 constexpr size_t kMaxDynSmem = 225 * 1024;   // dynamic shared memory per CTA
@@ -79,6 +81,21 @@ struct GemvArgs {
     unsigned flags;
     int C;
     int vsplit[kMaxCluster + 1];   // CTA j of a cluster: virtual panels [vsplit[j], vsplit[j+1])
+    // Grouped calls: up to kMaxGroup matrices of one format (N, K, g, nS, Ks)
+    // that read the same x.  Row blocks [rb_start[m], rb_start[m+1]) of the
+    // grid belong to matrix m, whose fields replace the ones above at entry.
+    int group;     // matrices in the call; 1: the fields above are the matrix
+    int rb_base;   // set at entry: the first row block of this CTA's matrix
+    int rb_start[kMaxGroup + 1];
+    struct Mat {
+        const uint8_t *planes;
+        const float *alpha_r, *alpha_c;
+        const uint8_t *s_planes;
+        const float *s_alpha_r, *s_alpha_c;
+        const uint32_t *s_idx;
+        float *y;
+        int M, M_pad, nchunks, pad;
+    } mats[kMaxGroup];
 };
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -442,19 +459,40 @@ __global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant
     // parallel copy into shared memory pays that latency once.
     __shared__ __align__(16) GemvArgs s_args;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    static_assert(sizeof(GemvArgs) % 4 == 0, "parameter block copied as words");
-    for (int i = tid; i < (int)(sizeof(GemvArgs) / 4); i += blockDim.x)
+    // (the per-matrix table of grouped calls stays in the parameter block)
+    static_assert(offsetof(GemvArgs, mats) % 4 == 0, "parameter block copied as words");
+    for (int i = tid; i < (int)(offsetof(GemvArgs, mats) / 4); i += blockDim.x)
         reinterpret_cast<int *>(&s_args)[i] = reinterpret_cast<const int *>(&args)[i];
     if (tid == 0) {
 #pragma unroll
         for (int s2 = 0; s2 < kSlots; ++s2) mbar_init(smem_addr(&s_bar[s2]));
         mbar_init_fence();
     }
+    if (args.group > 1) {   // a grouped call: this CTA's matrix
+        __syncthreads();
+        if (tid == 0) {
+            int m = 0;
+            while (m + 1 < s_args.group && (int)blockIdx.y >= s_args.rb_start[m + 1]) ++m;
+            const GemvArgs::Mat &mt = args.mats[m];
+            s_args.planes = mt.planes;
+            s_args.alpha_r = mt.alpha_r;
+            s_args.alpha_c = mt.alpha_c;
+            s_args.s_planes = mt.s_planes;
+            s_args.s_alpha_r = mt.s_alpha_r;
+            s_args.s_alpha_c = mt.s_alpha_c;
+            s_args.s_idx = mt.s_idx;
+            s_args.y = mt.y;
+            s_args.M = mt.M;
+            s_args.M_pad = mt.M_pad;
+            s_args.nchunks = mt.nchunks;
+            s_args.rb_base = s_args.rb_start[m];
+        }
+    }
     __syncthreads();
     const GemvArgs &a = s_args;
     cg::cluster_group cluster = cg::this_cluster();
     const int j = (int)cluster.block_rank();
-    const int rb = blockIdx.y, b = blockIdx.z;
+    const int rb = (int)blockIdx.y - a.rb_base, b = blockIdx.z;
     const int vb = a.vsplit[j], n_v = a.vsplit[j + 1] - a.vsplit[j];
     const int cpb = a.cpb, R = cpb * kChunkRows;
     const int c_first = rb * cpb;
@@ -845,35 +883,64 @@ extern "C" size_t fb_gemv_workspace_bytes(const fb_weights *W, int batch) {
     return 0;   // partial sums stay in the cluster's shared memory
 }
 
-extern "C" fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtype t, int batch, int ldx,
-                                     float *Y, int ldy, void *ws, size_t ws_bytes, unsigned flags,
-                                     void *stream) {
-    (void)ws;
-    (void)ws_bytes;
-    fb_status st = check_weights(W);
-    if (st != FB_OK) return st;
+// One launch for n matrices of one format that read the same X (n = 1: a
+// plain call).  Y[m] is matrix m's output with row stride ldy[m].
+static fb_status launch_gemv(const fb_weights *const *Ws, int n, const void *X, fb_dtype t, int batch, int ldx,
+                             float *const *Y, const int *ldy, unsigned flags, void *stream) {
+    const fb_weights *W = Ws[0];
     const int es = dtype_size(t);
-    if (!X || !Y || !es || batch < 1 || batch > kMaxBatch || ldx < W->N || ldy < W->M ||
-        (flags & ~kKnownFlags) || ((flags & FB_GEMV_INDEPENDENT) && !(flags & FB_GEMV_PDL)))
+    if (!X || !es || batch < 1 || batch > kMaxBatch || ldx < W->N || (flags & ~kKnownFlags) ||
+        ((flags & FB_GEMV_INDEPENDENT) && !(flags & FB_GEMV_PDL)))
         return FB_ERR_INVALID_VALUE;
-    if (!aligned(X, es) || !aligned(Y, 4)) return FB_ERR_MISALIGNED;
-
-    const Plan &pl = cached_plan(W, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0);
+    if (!aligned(X, es)) return FB_ERR_MISALIGNED;
+    int M_max = 0;
+    for (int m = 0; m < n; ++m) {
+        if (!Y[m] || ldy[m] < Ws[m]->M) return FB_ERR_INVALID_VALUE;
+        if (!aligned(Y[m], 4)) return FB_ERR_MISALIGNED;
+        M_max = std::max(M_max, Ws[m]->M);
+    }
+    // the plan of the largest matrix (the format, hence the panels, is shared)
+    fb_weights Wp = *W;
+    Wp.M = M_max;
+    const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0);
     const KernelFn fn = pick_kernel(t);
     if (!prepare_kernel(fn, pl.smem)) return FB_ERR_CUDA;
 
     GemvArgs a;
-    a.planes = (const uint8_t *)W->planes;
-    a.alpha_r = W->alpha_r;
-    a.alpha_c = W->alpha_c;
-    a.s_planes = (const uint8_t *)W->s_planes;
-    a.s_alpha_r = W->s_alpha_r;
-    a.s_alpha_c = W->s_alpha_c;
-    a.s_idx = W->s_idx;
+    a.group = n;
+    a.rb_base = 0;
+    a.rb_start[0] = 0;
+    for (int m = 0; m < kMaxGroup; ++m) {
+        GemvArgs::Mat &mt = a.mats[m];
+        const fb_weights *Wm = Ws[std::min(m, n - 1)];
+        mt.planes = (const uint8_t *)Wm->planes;
+        mt.alpha_r = Wm->alpha_r;
+        mt.alpha_c = Wm->alpha_c;
+        mt.s_planes = (const uint8_t *)Wm->s_planes;
+        mt.s_alpha_r = Wm->s_alpha_r;
+        mt.s_alpha_c = Wm->s_alpha_c;
+        mt.s_idx = Wm->s_idx;
+        mt.y = Y[std::min(m, n - 1)];
+        mt.M = Wm->M;
+        mt.M_pad = round_up(Wm->M, kChunkRows);
+        mt.nchunks = mt.M_pad / kChunkRows;
+        mt.pad = 0;
+        if (m < n) a.rb_start[m + 1] = a.rb_start[m] + ceil_div(mt.nchunks, pl.cpb);
+    }
+    for (int m = n; m < kMaxGroup; ++m) a.rb_start[m + 1] = a.rb_start[n];
+    const int rows_of_blocks = a.rb_start[n];
+    if (rows_of_blocks > 65535) return FB_ERR_UNSUPPORTED;
+    a.planes = a.mats[0].planes;
+    a.alpha_r = a.mats[0].alpha_r;
+    a.alpha_c = a.mats[0].alpha_c;
+    a.s_planes = a.mats[0].s_planes;
+    a.s_alpha_r = a.mats[0].s_alpha_r;
+    a.s_alpha_c = a.mats[0].s_alpha_c;
+    a.s_idx = a.mats[0].s_idx;
     a.x = X;
-    a.y = Y;
+    a.y = Y[0];
     a.M = W->M;
-    a.M_pad = pl.M_pad;
+    a.M_pad = a.mats[0].M_pad;
     a.N = W->N;
     a.K = W->K;
     a.nS = W->nS;
@@ -881,15 +948,15 @@ extern "C" fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtyp
     a.Ks = W->nS > 0 ? W->Ks : 0;
     a.Pg = pl.Pg;
     a.Ps = pl.Ps;
-    a.nchunks = pl.nchunks;
+    a.nchunks = a.mats[0].nchunks;
     a.cpb = pl.cpb;
     a.ldx = ldx;
-    a.ldy = ldy;
+    a.ldy = ldy[0];
     a.flags = flags;
     a.C = pl.C;
     std::copy(pl.vsplit, pl.vsplit + kMaxCluster + 1, a.vsplit);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(pl.C, pl.RB, batch);
+    cfg.gridDim = dim3(pl.C, rows_of_blocks, batch);
     cfg.blockDim = dim3(pl.nwarps * 32);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = as_stream(stream);
@@ -907,6 +974,35 @@ extern "C" fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtyp
     cfg.attrs = attr;
     cfg.numAttrs = na;
     return status_of(cudaLaunchKernelEx(&cfg, fn, a));
+}
+
+extern "C" fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtype t, int batch, int ldx,
+                                     float *Y, int ldy, void *ws, size_t ws_bytes, unsigned flags,
+                                     void *stream) {
+    (void)ws;
+    (void)ws_bytes;
+    const fb_status st = check_weights(W);
+    if (st != FB_OK) return st;
+    const fb_weights *Ws[1] = {W};
+    float *Ys[1] = {Y};
+    const int ldys[1] = {ldy};
+    return launch_gemv(Ws, 1, X, t, batch, ldx, Ys, ldys, flags, stream);
+}
+
+extern "C" fb_status fb_gemv_grouped(const fb_weights *const *W, int n, const void *x, fb_dtype t, float *const *y,
+                                     unsigned flags, void *stream) {
+    if (!W || !y || n < 1 || n > kMaxGroup) return FB_ERR_INVALID_VALUE;
+    int ldy[kMaxGroup];
+    for (int m = 0; m < n; ++m) {
+        const fb_status st = check_weights(W[m]);
+        if (st != FB_OK) return st;
+        const fb_weights *A = W[0], *B = W[m];
+        const int ksA = A->nS > 0 ? A->Ks : 0, ksB = B->nS > 0 ? B->Ks : 0;
+        if (B->N != A->N || B->K != A->K || B->g != A->g || B->nS != A->nS || ksB != ksA)
+            return FB_ERR_INVALID_VALUE;   // not one format
+        ldy[m] = B->M;
+    }
+    return launch_gemv(W, n, x, t, 1, W[0]->N, y, ldy, flags, stream);
 }
 
 extern "C" fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned flags, int sms, int *out) {

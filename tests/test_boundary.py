@@ -184,6 +184,25 @@ def test_launch_plan_rejects_bad_arguments(L):
     assert L.fb_device_errors(None, 0) == INVALID
 
 
+def test_grouped_rejects_bad_arguments(L):
+    def call(structs, n, x=FAKE, ys=None, flags=0):
+        arr = (C.POINTER(fb.FbWeightsStruct) * max(1, len(structs)))(*[C.pointer(s) for s in structs])
+        yp = (C.c_void_p * max(1, len(structs)))(*([FAKE] * len(structs) if ys is None else ys))
+        return L.fb_gemv_grouped(C.cast(arr, C.c_void_p), n, x, 1, C.cast(yp, C.c_void_p), flags, None)
+    a = fake_weights()
+    assert call([a, fake_weights(N=1024)], 2) == INVALID              # another N
+    assert call([a, fake_weights(K=3)], 2) == INVALID                 # another K
+    assert call([a, fake_weights(g=8)], 2) == INVALID                 # another g
+    assert call([a, fake_weights(nS=10, Ks=2)], 2) == INVALID         # another salient format
+    assert call([a] * 5, 5) == INVALID                                 # at most 4
+    assert call([a], 0) == INVALID
+    assert call([a, fake_weights(M=300)], 2, ys=[FAKE, None]) == INVALID
+    assert call([a, fake_weights(M=300)], 2, ys=[FAKE, FAKE + 2]) == MISALIGNED
+    assert call([a, fake_weights(M=300)], 2, flags=2) == INVALID       # INDEPENDENT needs PDL
+    assert call([a, fake_weights(planes=FAKE + 4)], 2) == MISALIGNED
+    assert L.fb_gemv_grouped(None, 1, FAKE, 1, None, 0, None) == INVALID
+
+
 def test_layout_spec_is_a_bijection():
     """Every (base, row, column) lands on its own bit of the packed buffer."""
     rng = np.random.default_rng(0)

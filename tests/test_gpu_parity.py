@@ -254,6 +254,64 @@ def test_invalid_salient_index_reads_nothing():
     assert fb.fb_validate_weights(Wu) == 1
 
 
+# --- grouped calls (several matrices of one format reading one x) ------------
+
+@pytest.mark.parametrize("flags", [0, 1, 3])
+def test_grouped_qkv_and_gate_up(flags):
+    """q, k, v of a 7B layer in one launch, and gate, up (another M) in one
+    launch; each result against the oracle with the shared x."""
+    for ms in ((0, 1, 2), (4, 5)):
+        ps = [wl.step7b_matrix(2, m) for m in ms]
+        for p in ps[1:]:
+            p.x = ps[0].x            # one x for the group
+        Ws = [fb.Weights.from_problem(p) for p in ps]
+        x = x_tensor(ps[0])[0]
+        ys = fb.fb_gemv_grouped(Ws, x, flags=flags)
+        torch.cuda.synchronize()
+        for p, y in zip(ps, ys):
+            check(p, y.cpu().numpy()[None].astype(np.float64), sample_rows(p.M, 96, 3))
+
+
+def test_grouped_equals_single_calls_and_ragged_rows():
+    """Matrices of different M (ragged last row blocks) in one launch give the
+    bits of separate calls with the same plan."""
+    ps = [wl.make_problem(M, 1280, 2, nS=45, Ks=2, x_dtype="f16", seed=40 + i) for i, M in enumerate((700, 33, 1000, 64))]
+    for p in ps[1:]:
+        p.x = ps[0].x
+    Ws = [fb.Weights.from_problem(p) for p in ps]
+    x = x_tensor(ps[0])[0]
+    ys = fb.fb_gemv_grouped(Ws, x)
+    torch.cuda.synchronize()
+    for p, y in zip(ps, ys):
+        check(p, y.cpu().numpy()[None].astype(np.float64))
+    one = fb.fb_gemv_grouped(Ws[:1], x)[0]
+    torch.cuda.synchronize()
+    assert torch.equal(one, ys[0])
+
+
+def test_grouped_in_graph_with_pdl():
+    ps = [wl.step7b_matrix(7, m) for m in (4, 5)]
+    ps[1].x = ps[0].x
+    Ws = [fb.Weights.from_problem(p) for p in ps]
+    x = x_tensor(ps[0])[0]
+    ys = [torch.full((p.M,), float("nan"), device=DEV) for p in ps]
+    s = torch.cuda.Stream()
+    flags = fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT
+    with torch.cuda.stream(s):
+        fb.fb_gemv_grouped(Ws, x, ys, flags=flags)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(3):
+                fb.fb_gemv_grouped(Ws, x, ys, flags=flags)
+    for y in ys:
+        y.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    for p, y in zip(ps, ys):
+        check(p, y.cpu().numpy()[None].astype(np.float64), sample_rows(p.M, 64, 9))
+
+
 # --- the five workloads ----------------------------------------------------------
 
 @pytest.mark.parametrize("integer_mode", [False, True])
