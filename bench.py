@@ -137,7 +137,8 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
                 "reasons": sorted(reasons), "samples": len(rows),
-                "power_w_max": max(r["power"] for r in rows)}
+                "power_w_max": max(r["power"] for r in rows),
+                "power_w_mean": round(statistics.mean(r["power"] for r in rows), 1)}
 
 
 def dist_setup(args):
@@ -383,6 +384,8 @@ def run_ours(args):
     if not args.no_7b:
         step7b = bench_7b(args, device, stream, world, peak)
     configs = None if args.no_configs else bench_configs(args, device, stream, world, peak)
+    ours_energy = round(clocks["power_w_mean"] * us_per_gemv, 2) if clocks and clocks.get("power_w_mean") else None
+    fp16 = None if args.no_configs else bench_fp16_dense(args, device, stream, world, gpu_id, us_per_gemv, ours_energy)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -404,6 +407,8 @@ def run_ours(args):
         "variants": {"g8_pair_tables": g8},
         "step_7b": step7b,
         "configs": configs,
+        "energy_uj_per_gemv": ours_energy,
+        "fp16_dense_comparator": fp16,
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 4),
                 "note": f"{n_e2e} eager fb_gemv calls per step from Python, pinned host x in and y out"},
@@ -537,6 +542,50 @@ def bench_configs(args, device, stream, world, peak):
         measure(f"layer70b_{M}x{N}_k3_g8", lambda i, si=si: wl.layer70b(si, 16) if i == 0 else
                 wl.make_problem(M, N, 3, g=8, nS=wl.salient_count(0.05, N), Ks=2, batch=16, x_dtype="f16",
                                 alpha_dist="small", seed=(7, si, i)), batches=wl.BATCHES70B)
+    return out
+
+
+def bench_fp16_dense(args, device, stream, world, gpu_id, ours_us, ours_energy_uj):
+    """The comparison the FluxBin page draws against uncompressed weights,
+    restated per GEMV on this GPU: a dense fp16 matrix-vector product
+    (torch.mv, i.e. cuBLAS) on the same shapes, with board energy per call
+    from the power sampled during its timed region."""
+    import torch
+    out = {}
+    for M, N in ((4096, 4096), (11008, 4096), (8192, 8192)):
+        per = M * N * 2
+        nsets = max(2, int(2 * 126e6 // per) + 1)
+        g = torch.Generator(device=device).manual_seed(M * 7 + N)
+        Ws = [torch.randn(M, N, device=device, dtype=torch.float16, generator=g) * 0.02 for _ in range(nsets)]
+        x = torch.randn(N, device=device, dtype=torch.float16, generator=g)
+        ys = [torch.empty(M, device=device, dtype=torch.float16) for _ in range(nsets)]
+        reps = max(1, 64 // nsets)
+
+        def body():
+            for _ in range(reps):
+                for W, y in zip(Ws, ys):
+                    torch.mv(W, x, out=y)
+        graph = capture(stream, body)
+        calls = reps * nsets
+        # about half a second of timed work, for the power samples
+        one, _ = time_graph(graph, stream, 3, 1, world)
+        n = max(10, int(500.0 / max(one / 3, 1e-3)))
+        sampler = ClockSampler(gpu_id)
+        ms, clocks = time_graph(graph, stream, n, args.warmup, world, sampler)
+        us = ms * 1e3 / (n * calls)
+        gbs = (per + 2 * N + 2 * M) / (us * 1e-6) / 1e9
+        e = {"us": round(us, 3), "gbs": round(gbs, 1), "weight_bytes": per}
+        if clocks and clocks.get("power_w_mean"):
+            e["energy_uj_per_gemv"] = round(clocks["power_w_mean"] * us, 2)
+        out[f"{M}x{N}"] = e
+        del graph, Ws, ys
+        torch.cuda.synchronize()
+    r = out["4096x4096"]
+    out["speedup_4096_ours_vs_fp16"] = round(r["us"] / ours_us, 2)
+    if ours_energy_uj and r.get("energy_uj_per_gemv"):
+        out["energy_ratio_4096_fp16_over_ours"] = round(r["energy_uj_per_gemv"] / ours_energy_uj, 2)
+    out["note"] = ("dense fp16 torch.mv (cuBLAS) on random weights of the same shapes, graph of calls over "
+                   "rotating copies larger than twice L2; energy = mean board power x time per call")
     return out
 
 

@@ -152,6 +152,18 @@ def test_gemv_batched_small(g):
     check(pi, run_gpu(pi))
 
 
+@pytest.mark.parametrize("batch", [2, 3, 16])
+@pytest.mark.parametrize("flags", [0, 3])
+def test_gemv_batched_tokens(batch, flags):
+    """Batched calls at full panels, narrow salient tails and both plans
+    (dependent and independent), odd and even batches."""
+    p = wl.make_problem(1000, 2304, 2, g=4, nS=300, Ks=2, x_dtype="f16", batch=batch, seed=50 + batch)
+    check(p, run_gpu(p, flags=flags))
+    pi = wl.make_problem(700, 1312, 3, g=8, nS=45, Ks=2, x_dtype="bf16", batch=batch, seed=60 + batch,
+                         integer_mode=True)
+    check(pi, run_gpu(pi, flags=flags))
+
+
 def test_gemv_batched_max_batch():
     p = wl.make_problem(40, 256, 1, g=4, x_dtype="f32", batch=64, seed=6)
     check(p, run_gpu(p))
