@@ -45,6 +45,7 @@
 #include <cstddef>
 #include <cstdio>
 #include <cstdlib>
+#include <mutex>
 #include <new>
 #include <type_traits>
 
@@ -833,17 +834,20 @@ const Plan &cached_plan(const fb_weights *W, int batch, int sms, bool independen
     return e.plan;
 }
 
-// Raise the kernel's dynamic shared-memory limit once per kernel and device.
+// Raise the kernel's dynamic shared-memory limit once per kernel and device
+// (callers may launch from several host threads: the record is locked).
 bool prepare_kernel(KernelFn fn, size_t smem) {
     struct Entry {
         KernelFn fn;
         int dev;
         size_t smem;
     };
+    static std::mutex lock;
     static Entry done[64];
     static int n_done = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> guard(lock);
     for (int i = 0; i < n_done; ++i)
         if (done[i].fn == fn && done[i].dev == dev && done[i].smem >= smem) return true;
     const size_t want = std::max<size_t>(smem, 100 * 1024);
