@@ -170,11 +170,18 @@ FB_API size_t fb_gemv_workspace_bytes(const fb_weights *W, int batch);
                           kernel still completes only after the previous one,
                           so ordering with later work is unchanged. */
 
+#define FB_GEMV_TEST_WAIT_TIMEOUT 0x80000000u /* for tests of the failure path:
+                          the kernel issues no weight copy, so its bounded wait
+                          for one runs out (about 0.2 s); it then writes NaN
+                          into every row and raises bit 0 of fb_device_errors.
+                          The context stays usable. */
+
 /* fb_gemv: y[i] = sum_j W_hat[i][j] * x[j] for i < M (batch 1), fp32 out,
  * overwriting y (beta = 0).  x: N elements of type t (2- or 4-byte aligned);
  * y: M floats, 4-byte aligned, must not alias x; ws: see
- * fb_gemv_workspace_bytes.  flags: 0 or FB_GEMV_PDL [| FB_GEMV_INDEPENDENT];
- * anything else is FB_ERR_INVALID_VALUE.  Table entries and all sums are
+ * fb_gemv_workspace_bytes.  flags: 0 or FB_GEMV_PDL [| FB_GEMV_INDEPENDENT],
+ * optionally | FB_GEMV_TEST_WAIT_TIMEOUT; anything else is
+ * FB_ERR_INVALID_VALUE.  Table entries and all sums are
  * fp32.  Deterministic: the same inputs give the same bits on every run.
  * Weight copies are waited for with a bound (about 0.2 s); a kernel that
  * gives up writes NaN into the rows it owns and raises bit 0 of

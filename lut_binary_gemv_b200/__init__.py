@@ -21,7 +21,7 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "FbError", "Weights", "lib", "library_path", "FB_GEMV_PDL", "FB_GEMV_INDEPENDENT",
+    "FbError", "Weights", "lib", "library_path", "FB_GEMV_PDL", "FB_GEMV_INDEPENDENT", "FB_GEMV_TEST_WAIT_TIMEOUT",
     "fb_packed_words", "fb_pack", "fb_pack_bits", "fb_unpack", "fb_vcm_gather",
     "fb_lut_build", "fb_validate_weights", "fb_gemv_workspace_bytes", "fb_gemv",
     "fb_gemv_batched", "fb_status_string", "fb_gemv_launch_plan", "fb_gemv_grouped", "fb_device_errors",
@@ -33,6 +33,7 @@ library_path = os.path.join(_HERE, "libfluxbin.so")
 FB_OK = 0
 FB_GEMV_PDL = 1
 FB_GEMV_INDEPENDENT = 2
+FB_GEMV_TEST_WAIT_TIMEOUT = 0x80000000
 _DTYPES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 _STATUS = {0: "FB_OK", 1: "FB_ERR_INVALID_VALUE", 2: "FB_ERR_UNSUPPORTED", 3: "FB_ERR_MISALIGNED",
            4: "FB_ERR_WORKSPACE", 5: "FB_ERR_CUDA"}

@@ -27,12 +27,6 @@ __host__ __device__ inline int panel_width(int N, int p) {
     return w < kPanelCols ? w : kPanelCols;
 }
 
-// Byte offset of (base k, panel p, chunk c) in a planes buffer.
-__host__ __device__ inline size_t block_offset(int k, int p, int c, int M_pad, int N) {
-    const int Bp = panel_width(N, p) / 8;
-    return (size_t)k * M_pad * (size_t)(N / 8) + (size_t)32 * p * M_pad + (size_t)32 * Bp * c;
-}
-
 // Byte offset, inside a chunk block, of stored position u of lane l.
 __host__ __device__ inline int position_offset(int u, int l, int Bp) {
     return (Bp % 16 == 0) ? (u / 16) * 512 + 16 * l + (u % 16) : (u / 4) * 128 + 4 * l + (u % 4);

@@ -45,8 +45,8 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_binding_constants_match_header():
     text = open(HEADER).read()
-    defines = dict((n, int(v)) for n, v in re.findall(r"#define\s+(FB_GEMV_\w+)\s+(\d+)u", text))
-    assert defines, "no launch flags found in the header"
+    defines = dict((n, int(v, 0)) for n, v in re.findall(r"#define\s+(FB_GEMV_\w+)\s+(0x[0-9a-fA-F]+|\d+)u", text))
+    assert len(defines) == 3, f"launch flags found in the header: {sorted(defines)}"
     for name, value in defines.items():
         assert getattr(fb, name) == value, name
     enums = dict((n, int(v)) for n, v in re.findall(r"\b(FB_(?:OK|ERR_\w+))\s*=\s*(\d+)", text))

@@ -385,3 +385,21 @@ def test_device_error_flags_stay_clear():
     W = fb.Weights.from_problem(p)
     fb.fb_gemv(W, torch.from_numpy(p.x[0]).cuda(), flags=fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT)
     assert fb.fb_device_errors(clear=True) == 0
+
+
+def test_bounded_wait_runs_out_and_reports():
+    """The failure path of the weight-copy waits: with no copy issued, each
+    wait gives up after its bound, the rows come back NaN, the device error
+    flag is raised, and the next call on the same context is correct."""
+    p = wl.make_problem(96, 512, 1, g=4, x_dtype="f32", seed=70)
+    W = fb.Weights.from_problem(p)
+    x = x_tensor(p)[0]
+    assert fb.fb_device_errors(clear=True) == 0
+    y = fb.fb_gemv(W, x, flags=fb.FB_GEMV_TEST_WAIT_TIMEOUT)
+    torch.cuda.synchronize()
+    assert torch.isnan(y).all()
+    assert fb.fb_device_errors(clear=True) == 1
+    assert fb.fb_device_errors(clear=True) == 0
+    check(p, run_gpu(p, W=W))
+    assert fb.fb_device_errors(clear=True) == 0
+
