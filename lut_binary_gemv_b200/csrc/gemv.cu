@@ -11,7 +11,8 @@
 // chunks; CTA j of the cluster takes a contiguous, balanced slice of the V
 // virtual panels, so the cluster covers every column of its rows.
 //
-// Per CTA (16 warps; warp w owns chunks w and w+16 of the row block):
+// Per CTA (16 warps, or 8 for dependent calls; warp w owns chunks w and
+// w + warps of the row block):
 //   1. before the programmatic-launch wait: the weights of the first panels
 //      start streaming into shared-memory slots (one bulk asynchronous copy
 //      per panel of the row block, completion on an mbarrier), and the row
@@ -58,8 +59,16 @@ namespace {
 
 constexpr int kMaxCluster = 8;
 constexpr int kMaxGroup = 4;            // matrices in one grouped call
-constexpr int kNW = 16;                 // warps per CTA
-constexpr int kMaxCpb = 32;             // chunks per row block (four per warp)
+// Two CTA shapes.  16 warps, one CTA per SM, up to 32 chunks per row block
+// and three weight slots: calls flagged independent (fewest table builds per
+// row).  8 warps, two CTAs per SM, up to 16 chunks and two slots: dependent
+// calls (twice the CTAs in one wave, shorter panel lists per CTA).  Both give
+// each warp two chunks of every panel.
+template <int NW>
+struct Shape {
+    static constexpr int kSlots = NW == 16 ? 3 : 2;
+    static constexpr int kMinBlocks = 16 / NW;     // CTAs per SM the registers allow
+};
 constexpr size_t kMaxDynSmem = 225 * 1024;   // dynamic shared memory per CTA
 constexpr size_t kSmemPerSM = 228 * 1024;
 constexpr size_t kStaticSmem = 1024;          // the kernel's static shared memory, rounded up
@@ -382,9 +391,10 @@ __device__ __forceinline__ void lookup_rows2(const uint32_t (&wa)[8], const uint
 // tables of the group's low and high 4 columns, each (+-z0 +- z1) + (+-z2 +-
 // z3).  Columns past a narrow panel's width have z = 0, so their entries are
 // 0.  T points at the buffer (entry b of group q at T[b*64 + q]).  Each of
-// the kNW warps writes 256 / kNW consecutive entries b of every group.
+// the NW warps writes 256 / NW consecutive entries b of every group.
+template <int NW>
 __device__ __forceinline__ void build_byte_table(const float *zp, float *T, int warp, int lane) {
-    constexpr int kHi = 16 / kNW;   // high-nibble values per warp: entries b = 16*kHi*warp ...
+    constexpr int kHi = 16 / NW;   // high-nibble values per warp: entries b = 16*kHi*warp ...
     const float4 za = *reinterpret_cast<const float4 *>(zp + 8 * lane);
     const float4 zb = *reinterpret_cast<const float4 *>(zp + 8 * lane + 4);
     float lo[16];
@@ -441,11 +451,11 @@ __device__ __forceinline__ void read_item_full(const uint8_t *slot, int lane, ui
 // row partials [R] | cluster inbox [R + C].
 constexpr int kTableBytes = 65536;
 constexpr int kZBytes = 2 * kPanelCols * 4;
-constexpr int kSlots = 3;
-constexpr int kItemsPerWarp = kMaxCpb / kNW;
+constexpr int kItemsPerWarp = 2;
 
-template <int XT>
-__global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant__ GemvArgs args) {
+template <int XT, int NW>
+__global__ void __launch_bounds__(NW * 32, Shape<NW>::kMinBlocks) gemv_kernel(const __grid_constant__ GemvArgs args) {
+    constexpr int kNW = NW, kSlots = Shape<NW>::kSlots;
     extern __shared__ __align__(128) float smem_f[];
     __shared__ __align__(8) unsigned long long s_bar[kSlots];
     // The launch's parameter block is new to every SM's constant cache, and the
@@ -584,7 +594,7 @@ __global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant
         }
         if (tid == 0 && ok) pending &= ~(1u << sl);
         float *tb = tables + 32 * buf;
-        build_byte_table(zbuf + buf * kPanelCols, tb, warp, lane);
+        build_byte_table<NW>(zbuf + buf * kPanelCols, tb, warp, lane);
         if (vi + 1 < n_v && tid < kPanelCols)   // z of the next panel into the other buffer
             zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
         if (vi + 3 < n_v) stage(st[buf ^ 1], s_desc[vi + 3], true);
@@ -678,9 +688,12 @@ __global__ void __launch_bounds__(kNW * 32, 1) gemv_kernel(const __grid_constant
 
 using KernelFn = void (*)(GemvArgs);
 
-KernelFn pick_kernel(fb_dtype t) {
-    return t == FB_F32 ? gemv_kernel<FB_F32> : t == FB_F16 ? gemv_kernel<FB_F16> : gemv_kernel<FB_BF16>;
+template <int NW>
+KernelFn pick_xt(fb_dtype t) {
+    return t == FB_F32 ? gemv_kernel<FB_F32, NW> : t == FB_F16 ? gemv_kernel<FB_F16, NW> : gemv_kernel<FB_BF16, NW>;
 }
+
+KernelFn pick_kernel(fb_dtype t, int nw) { return nw == 16 ? pick_xt<16>(t) : pick_xt<8>(t); }
 
 fb_status check_weights(const fb_weights *W) {
     if (!W || !valid_dims(W->K, W->M, W->N) || !(W->g == 1 || W->g == 2 || W->g == 4 || W->g == 8))
@@ -723,20 +736,23 @@ void split_panels(int V, int C, int *vsplit, int *max_n) {
 // Dynamic shared memory of a CTA with cpb chunks of rows and KB bases:
 // tables, z, rings, row scales, row partials and the inbox of row partials
 // pushed by the cluster (C * ceil(R / C) <= R + C floats).
-size_t smem_for(int cpb, int KB, int nv) {
+size_t smem_for(int cpb, int KB, int nv, int nw) {
     const size_t R = (size_t)cpb * kChunkRows;
-    return (size_t)kTableBytes + kZBytes + (size_t)kSlots * cpb * 1024 + R * KB * 4 + R * 4 +
+    const int slots = nw == 16 ? Shape<16>::kSlots : Shape<8>::kSlots;
+    return (size_t)kTableBytes + kZBytes + (size_t)slots * cpb * 1024 + R * KB * 4 + R * 4 +
            ((R + kMaxCluster + 1) & ~(size_t)1) * 4 + (size_t)nv * sizeof(PanelDesc);
 }
 
 // The launch plan: cluster size C (the split of the V virtual panels over
 // the cluster's CTAs) and row block size (cpb chunks of 32 rows).
-//  * Calls flagged independent overlap their neighbours, so the plan that
-//    does the least work wins: the largest row blocks (fewest table builds
-//    per row), C = 2 for matrices of at most 8 row blocks, else 1.
-//  * A dependent call is timed alone: its latency is about a fixed 4 us plus
-//    1.2 us per panel a CTA works through (build, barrier, lookups), times
-//    the number of waves; more CTAs per cluster shorten a CTA's panel list.
+//  * Calls flagged independent (16-warp CTAs) overlap their neighbours, so
+//    the plan that does the least work wins: the largest row blocks (fewest
+//    table builds per row), C = 2 for matrices of at most 8 row blocks,
+//    else 1.
+//  * A dependent call (8-warp CTAs, two per SM) is timed alone: its latency
+//    is about a fixed 4 us plus 1.2 us per panel a CTA works through (build,
+//    barrier, lookups), times the number of waves; more CTAs per cluster
+//    shorten a CTA's panel list.
 // Both rules were fitted to timings of this kernel on B200.
 Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
     Plan pl;
@@ -746,44 +762,47 @@ Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
     pl.Ps = W->nS > 0 ? num_panels(pl.nS_pad) : 0;
     pl.V = pl.Pg * W->K + pl.Ps * (W->nS > 0 ? W->Ks : 0);
     pl.nchunks = pl.M_pad / kChunkRows;
-    pl.nwarps = kNW;
+    const int nw = independent ? 16 : 8, max_cpb = 2 * nw;   // the CTA shape (Shape<NW>)
+    pl.nwarps = nw;
     const int KB = W->K + (W->nS > 0 ? W->Ks : 0);
-    const int occ_regs = 65536 / (kNW * 32 * 128);   // CTAs per SM by registers (128 per thread)
+    const int occ_regs = 65536 / (nw * 32 * 128);   // CTAs per SM by registers (128 per thread)
     auto fits = [&](int C, int cpb) {
         int vs[kMaxCluster + 1], nvm;
         split_panels(pl.V, C, vs, &nvm);
-        return smem_for(cpb, KB, nvm) <= kMaxDynSmem;
+        return smem_for(cpb, KB, nvm, nw) <= kMaxDynSmem;
     };
     auto set = [&](int C, int cpb) {
         pl.C = C;
         pl.RB = ceil_div(pl.nchunks, cpb);
-        pl.cpb = ceil_div(pl.nchunks, pl.RB);   // balanced: the same rows, less padding
+        // independent plans balance the row blocks (the same rows, less padding)
+        pl.cpb = independent ? ceil_div(pl.nchunks, pl.RB) : cpb;
         int nvm;
         split_panels(pl.V, C, pl.vsplit, &nvm);
     };
     if (independent) {
-        int cpb = std::min(kMaxCpb, pl.nchunks);
+        int cpb = std::min(max_cpb, pl.nchunks);
         while (cpb > 1 && !fits(2, cpb)) --cpb;
         const int RB = ceil_div(pl.nchunks, cpb);
         set(std::min(pl.V, RB <= 8 ? 2 : 1), cpb);
     } else {
         const double fixed = 4.0, per_panel = 1.2, per_item = 0.1;   // microseconds
         double best = 1e300;
-        set(1, std::min(kMaxCpb, pl.nchunks));
+        set(1, std::min(max_cpb, pl.nchunks));
         for (int C = 1; C <= std::min(kMaxCluster, pl.V); ++C) {
             int vs[kMaxCluster + 1], nvm;
             split_panels(pl.V, C, vs, &nvm);
-            // at least one chunk per warp (fewer measured slower on B200)
-            for (int cpb = std::min(kNW, pl.nchunks); cpb <= std::min(kMaxCpb, pl.nchunks); ++cpb) {
+            // whole chunks per warp (uneven splits measured slower on B200), or
+            // the whole matrix when it has fewer chunks than warps
+            for (int cpb = std::min(nw, pl.nchunks); cpb <= std::min(max_cpb, pl.nchunks);
+                 cpb += (pl.nchunks < nw ? max_cpb : nw)) {
                 const int RB = ceil_div(pl.nchunks, cpb);
                 if (RB > 65535) continue;
-                if (cpb > 1 && ceil_div(pl.nchunks, cpb - 1) == RB) continue;   // same split, fewer rows
-                const size_t smem = smem_for(cpb, KB, nvm);
+                const size_t smem = smem_for(cpb, KB, nvm, nw);
                 if (smem > kMaxDynSmem) continue;
                 const int occ = std::max(1, std::min(occ_regs, (int)(kSmemPerSM / (smem + kStaticSmem + 1024))));
                 const long ctas = (long)C * RB * batch;
                 const double waves = std::ceil((double)ctas / ((double)sms * occ));
-                const double cost = waves * (fixed + nvm * (per_panel + std::ceil((double)cpb / kNW) * per_item));
+                const double cost = waves * (fixed + nvm * (per_panel + std::ceil((double)cpb / nw) * per_item));
                 if (cost < best * 0.999) {
                     best = cost;
                     set(C, cpb);
@@ -797,16 +816,16 @@ Plan make_plan(const fb_weights *W, int batch, int sms, bool independent) {
         int oc = 0, ocpb = 0;
         if (sscanf(ov, "%d,%d", &oc, &ocpb) == 2 && oc >= 1 && ocpb >= 1) {
             pl.C = std::min(std::min(oc, kMaxCluster), pl.V);
-            pl.cpb = std::min(std::min(ocpb, kMaxCpb), pl.nchunks);
+            pl.cpb = std::min(std::min(ocpb, max_cpb), pl.nchunks);
             int nvm;
             split_panels(pl.V, pl.C, pl.vsplit, &nvm);
-            while (pl.cpb > 1 && smem_for(pl.cpb, KB, nvm) > kMaxDynSmem) --pl.cpb;
+            while (pl.cpb > 1 && smem_for(pl.cpb, KB, nvm, nw) > kMaxDynSmem) --pl.cpb;
             pl.RB = ceil_div(pl.nchunks, pl.cpb);
         }
     }
     int nv_max = 0;
     for (int jj = 0; jj < pl.C; ++jj) nv_max = std::max(nv_max, pl.vsplit[jj + 1] - pl.vsplit[jj]);
-    pl.smem = smem_for(pl.cpb, KB, nv_max);
+    pl.smem = smem_for(pl.cpb, KB, nv_max, nw);
     return pl;
 }
 
@@ -901,7 +920,7 @@ static fb_status launch_gemv(const fb_weights *const *Ws, int n, const void *X, 
     fb_weights Wp = *W;
     Wp.M = M_max;
     const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0);
-    const KernelFn fn = pick_kernel(t);
+    const KernelFn fn = pick_kernel(t, pl.nwarps);
     if (!prepare_kernel(fn, pl.smem)) return FB_ERR_CUDA;
 
     GemvArgs a;
