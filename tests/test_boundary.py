@@ -174,6 +174,19 @@ def test_launch_plan_covers_the_matrix(L, shape, batch, flags):
     assert 0 < plan["smem"] <= 225 * 1024
 
 
+def test_launch_plan_shapes_by_call_kind(L):
+    """Calls flagged independent get the 16-warp CTA (row blocks of up to 32
+    chunks); dependent calls the 8-warp CTA (up to 16 chunks, a whole number
+    of chunks per warp when the matrix has enough)."""
+    for M, N, K, g, nS, Ks in ((4096, 4096, 2, 4, 128, 2), (11008, 4096, 2, 4, 123, 2), (8192, 8192, 3, 8, 410, 2)):
+        s = fake_weights(M=M, N=N, K=K, g=g, nS=nS, Ks=Ks)
+        ind = fb.fb_gemv_launch_plan(s, 1, 3, 148)
+        dep = fb.fb_gemv_launch_plan(s, 1, 1, 148)
+        assert ind["warps"] == 16 and ind["cpb"] <= 32
+        assert dep["warps"] == 8 and dep["cpb"] <= 16 and dep["cpb"] % 8 == 0
+        assert dep["C"] * dep["RB"] <= 2 * 148        # one wave at two CTAs per SM
+
+
 def test_launch_plan_rejects_bad_arguments(L):
     s = fake_weights()
     out = (C.c_int * 6)()
