@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile", action="store_true",
                     help="small case for ncu: 32 weight sets (142 MB), one pass per step, headline graph only")
+    ap.add_argument("--dependent", action="store_true",
+                    help="with --profile: the graph as a dependent chain (the dependent-call plan)")
     return ap.parse_args()
 
 
@@ -320,7 +322,7 @@ def run_ours(args):
         return body
 
     gemvs = WEIGHT_SETS * PASSES_PER_STEP
-    graph = capture(stream, step(Ws, indep))
+    graph = capture(stream, step(Ws, fb.FB_GEMV_PDL if (args.profile and args.dependent) else indep))
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_id = vis.split(",")[local] if vis else str(local)
     sampler = ClockSampler(gpu_id)
