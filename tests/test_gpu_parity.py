@@ -132,11 +132,38 @@ SMALL = [
 @pytest.mark.parametrize("g", [1, 2, 4, 8])
 @pytest.mark.parametrize("shape", SMALL, ids=[f"{s[0]}x{s[1]}k{s[2]}s{s[3]}{s[5]}" for s in SMALL])
 @pytest.mark.parametrize("integer_mode", [False, True])
-def test_gemv_small(g, shape, integer_mode):
+@pytest.mark.parametrize("flags", [0, 3], ids=["dependent", "independent"])   # both CTA shapes
+def test_gemv_small(g, shape, integer_mode, flags):
     M, N, K, nS, Ks, dt = shape
     p = wl.make_problem(M, N, K, g=g, nS=nS, Ks=Ks, x_dtype=dt, alpha_dist="unit",
-                        seed=hash(shape) % 997 + g, integer_mode=integer_mode)
+                        seed=(M * 31 + N * 7 + K * 3 + nS) % 997 + g, integer_mode=integer_mode)
+    check(p, run_gpu(p, flags=flags))
+
+
+@pytest.mark.parametrize("flags", [0, 3], ids=["dependent", "independent"])
+def test_gemv_maximum_rows(flags):
+    """M = 2^24 rows (the largest M the ABI takes), one 32-column panel."""
+    p = wl.make_problem(1 << 24, 32, 1, g=4, x_dtype="f16", seed=80)
+    check(p, run_gpu(p, flags=flags), sample_rows(p.M, 128, 80))
+
+
+@pytest.mark.parametrize("flags", [0, 3], ids=["dependent", "independent"])
+def test_gemv_maximum_columns(flags):
+    """N = 2^20 columns (the largest N the ABI takes): 4096 panels, 1000
+    salient columns."""
+    p = wl.make_problem(64, 1 << 20, 1, g=8, nS=1000, Ks=1, x_dtype="bf16", seed=81)
+    check(p, run_gpu(p, flags=flags))
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF], ids=["all_minus", "all_plus"])
+def test_gemv_constant_signs(fill):
+    """Every weight -1 (or +1): each row is -(or +) alpha_r times the
+    alpha_c-weighted sum of x; integer mode makes it exact."""
+    p = wl.make_problem(300, 1056, 2, g=4, nS=70, Ks=2, x_dtype="f16", seed=82, integer_mode=True)
+    p.sign_bits[...] = fill
+    p.s_sign_bits[...] = fill
     check(p, run_gpu(p))
+    check(p, run_gpu(p, flags=3))
 
 
 def test_gemv_alpha_c_none():
