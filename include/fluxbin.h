@@ -216,7 +216,10 @@ FB_API fb_status fb_gemv_grouped(const fb_weights *const *W, int n, const void *
  * block, out[2] = row blocks, out[3] = warps per CTA, out[4] = dynamic shared
  * memory bytes per CTA, out[5] = virtual panels (256-column panels x bases).
  * out must hold 6 ints.  Returns FB_OK, or FB_ERR_INVALID_VALUE for invalid
- * weights, batch, sms or flags. */
+ * weights, batch, sms or flags.  Tuning aid: the environment variable
+ * FB_PLAN="C,cpb", read when a plan is first made for a shape, forces the
+ * cluster size and row block (clamped to what the matrix and shared memory
+ * allow). */
 FB_API fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned flags, int sms, int *out);
 
 /* fb_device_errors: synchronises the current device, then stores in *flags
