@@ -16,8 +16,10 @@ timed too and reported as "dependent_chain".
 Printed: one JSON line (rank 0).  value = achieved GB/s of algorithmic bytes
 (packed planes, scales, salient data, x, y) over all ranks; also GEMV us, the
 g = 8 variant on the same weights, the 7B-shaped decode step (224 GEMVs), the
-roofline of the GEMV kernel against the measured HBM peak, e2e through the
-Python API with host buffers, and the fp64 CPU oracle as baseline.
+roofline of the GEMV kernel against the measured HBM peak, every workload at
+its own shape, a dense fp16 comparator with energy per call, e2e through the
+public API with pinned host buffers copied in and out every step (graph-replayed
+and eager calls), and the fp64 CPU oracle as baseline.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -355,31 +357,51 @@ def run_ours(args):
     g8_dep = side(Wg, fb.FB_GEMV_PDL)
     g8["dependent_chain_gemv_us"] = g8_dep["gemv_us"]
 
-    # e2e through the Python API: host x in, host y out, every step
+    # e2e through the public API, every step: the step's x copied in from
+    # pinned host memory, its 64 fb_gemv calls (independent calls, replayed
+    # from a captured CUDA graph), its y read back into pinned host memory.
+    # The same with 64 eager Python calls per step is reported beside it.
     n_e2e = WEIGHT_SETS
     x_host = torch.stack([x.cpu() for x in xs]).pin_memory()
     y_host = torch.empty((n_e2e, 4096), dtype=torch.float32).pin_memory()
     x_dev = torch.empty_like(x_host, device=device)
     y_dev = torch.empty((n_e2e, 4096), dtype=torch.float32, device=device)
     e2e_steps = max(10, args.steps // 10)
-    with torch.cuda.stream(stream):
-        def e2e_step():
-            x_dev.copy_(x_host, non_blocking=True)
-            for r in range(n_e2e):
-                fb.fb_gemv(Ws[r], x_dev[r], y=y_dev[r])
-            y_host.copy_(y_dev, non_blocking=True)
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
-        barrier(world)
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        s1.record(stream)
-        s1.synchronize()
-    ms_e2e = max_over_ranks(s0.elapsed_time(s1), world)
-    e2e_gbs = bytes_per * n_e2e * e2e_steps / (ms_e2e * 1e-3) / 1e9 * world
+
+    def e2e_run(step_fn, steps):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                step_fn()
+            torch.cuda.synchronize()
+            barrier(world)
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(steps):
+                step_fn()
+            s1.record(stream)
+            s1.synchronize()
+        ms_e = max_over_ranks(s0.elapsed_time(s1), world)
+        return bytes_per * n_e2e * steps / (ms_e * 1e-3) / 1e9 * world
+
+    def gemvs_e2e():
+        for r in range(n_e2e):
+            fb.fb_gemv(Ws[r], x_dev[r], y=y_dev[r], flags=indep)
+    g_e2e = capture(stream, gemvs_e2e)
+
+    def graph_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        g_e2e.replay()
+        y_host.copy_(y_dev, non_blocking=True)
+
+    def eager_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        for r in range(n_e2e):
+            fb.fb_gemv(Ws[r], x_dev[r], y=y_dev[r])
+        y_host.copy_(y_dev, non_blocking=True)
+
+    e2e_gbs = e2e_run(graph_step, e2e_steps)
+    e2e_eager_gbs = e2e_run(eager_step, e2e_steps)
+    del g_e2e
     torch.cuda.synchronize()
 
     step7b = None
@@ -413,7 +435,10 @@ def run_ours(args):
         "fp16_dense_comparator": fp16,
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 4),
-                "note": f"{n_e2e} eager fb_gemv calls per step from Python, pinned host x in and y out"},
+                "note": (f"per step: pinned host x ({n_e2e} x 4096 fp16) copied in, {n_e2e} fb_gemv calls "
+                         "(PDL + FB_GEMV_INDEPENDENT, replayed from a CUDA graph), y read back to pinned host")},
+        "e2e_eager": {"value": round(e2e_eager_gbs, 2), "unit": "GB/s",
+                      "note": f"the same with {n_e2e} eager Python fb_gemv calls per step (dependent-call plan)"},
         "gpu_launches": args.steps * gemvs,
         "clocks": clocks,
         "cpu_baseline": cpu,
