@@ -550,11 +550,24 @@ __global__ void __launch_bounds__(NW * 32, Shape<NW>::kMinBlocks) gemv_kernel(co
     auto z_of = [&](const Staged &t) { return t.xi >= 0 ? __fmul_rn(t.ac, x_value<XT>(t.x)) : 0.0f; };
     if (n_v > 0) stage(st[0], panel_desc(a, vb), independent);
     griddep_launch_dependents();
-    // the row block's row scales, every base (rows past M: 0)
-    for (int t = tid; t < KB * R; t += blockDim.x) {
-        const int kb = t / R, r = t - kb * R, row = c_first * kChunkRows + r;
-        const float *src = kb < a.K ? a.alpha_r + (size_t)kb * a.M : a.s_alpha_r + (size_t)(kb - a.K) * a.M;
-        s_ar[t] = row < a.M ? __ldg(src + row) : 0.0f;
+    // the row block's row scales, every base (rows past M: 0); a thread's
+    // loads are issued in batches of kArBatch before any is stored, so they
+    // cost one memory latency per batch rather than one each
+    constexpr int kArBatch = 8;
+    for (int t0 = 0; t0 < KB * R; t0 += kArBatch * (int)blockDim.x) {
+        float v[kArBatch];
+#pragma unroll
+        for (int u = 0; u < kArBatch; ++u) {
+            const int t = t0 + u * (int)blockDim.x + tid;
+            const int kb = t / R, r = t - kb * R, row = c_first * kChunkRows + r;
+            const float *src = kb < a.K ? a.alpha_r + (size_t)kb * a.M : a.s_alpha_r + (size_t)(kb - a.K) * a.M;
+            v[u] = t < KB * R && row < a.M ? __ldg(src + row) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kArBatch; ++u) {
+            const int t = t0 + u * (int)blockDim.x + tid;
+            if (t < KB * R) s_ar[t] = v[u];
+        }
     }
 
     // ---- 2. activations (may be the previous kernel's output) --------------
