@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
     FB_OK = 0,
     FB_ERR_INVALID_VALUE = 1, /* a size, pointer, dtype or group width is invalid */
-    FB_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+    FB_ERR_UNSUPPORTED = 2,   /* valid request outside what this library implements */
     FB_ERR_MISALIGNED = 3,    /* a pointer breaks the alignment stated below */
     FB_ERR_WORKSPACE = 4,     /* workspace missing, misaligned or too small */
     FB_ERR_CUDA = 5           /* the CUDA runtime reported an error */
