@@ -289,3 +289,24 @@ def layer70b(shape_index: int, batch: int, integer_mode: bool = False) -> Proble
 
 def all_named() -> List[str]:
     return ["tiny", "layer4096", "ternary11008", "step7b", "layer70b"]
+
+
+@dataclasses.dataclass
+class FitInputs:
+    """A dense matrix to decompose and calibration activations for the
+    saliency proxy (inputs of the fitter, the step before the GEMV)."""
+
+    W: np.ndarray   # float32 [M][N]
+    X: np.ndarray   # float32 [T][N]
+
+
+def fit_inputs(M: int, N: int, T: int = 64, seed=7) -> FitInputs:
+    """A dense LLaMA-like layer W ~ N(0, 0.02^2) and activations with outlier
+    channels: X[t][j] = s_j * N(0, 1), s_j = exp(N(0, 1)) (a few columns carry
+    much larger activations, which is what makes some columns salient).  Draw
+    order: W, s, X."""
+    rng = np.random.default_rng(seed)
+    W = rng.normal(0.0, 0.02, size=(M, N)).astype(np.float32)
+    s = np.exp(rng.normal(0.0, 1.0, size=N))
+    X = (rng.normal(0.0, 1.0, size=(T, N)) * s).astype(np.float32)
+    return FitInputs(W=W, X=X)
