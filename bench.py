@@ -410,6 +410,7 @@ def run_ours(args):
     configs = None if args.no_configs else bench_configs(args, device, stream, world, peak)
     ours_energy = round(clocks["power_w_mean"] * us_per_gemv, 2) if clocks and clocks.get("power_w_mean") else None
     fp16 = None if args.no_configs else bench_fp16_dense(args, device, stream, world, gpu_id, us_per_gemv, ours_energy)
+    fitter = None if args.no_configs else bench_fit(args, device, stream, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -433,6 +434,7 @@ def run_ours(args):
         "configs": configs,
         "energy_uj_per_gemv": ours_energy,
         "fp16_dense_comparator": fp16,
+        "fitter": fitter,
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 4),
                 "note": (f"per step: pinned host x ({n_e2e} x 4096 fp16) copied in, {n_e2e} fb_gemv calls "
@@ -569,6 +571,53 @@ def bench_configs(args, device, stream, world, peak):
         measure(f"layer70b_{M}x{N}_k3_g8", lambda i, si=si: wl.layer70b(si, 16) if i == 0 else
                 wl.make_problem(M, N, 3, g=8, nS=wl.salient_count(0.05, N), Ks=2, batch=16, x_dtype="f16",
                                 alpha_dist="small", seed=(7, si, i)), batches=wl.BATCHES70B)
+    return out
+
+
+def bench_fit(args, device, stream, peak):
+    """The fitter on a 4096 x 4096 layer (K = 2, 128 salient columns with Ks =
+    2, 8 alternating sweeps, 64 calibration rows): ms per whole fit on the
+    GPU, and the bytes its passes over the residual must move."""
+    import torch
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    M = N = 4096
+    K, Ks, nS, sweeps, T = 2, 2, 128, 8, 64
+    fi = wl.fit_inputs(M, N, T=T, seed=21)
+    W = torch.from_numpy(fi.W).to(device)
+    X = torch.from_numpy(fi.X).to(device)
+    nS_pad = (nS + 31) // 32 * 32
+    per_base = lambda m, n: (8 * sweeps + 9) * m * n        # 2 passes per sweep + read/write R + signs
+    nbytes = (8 * M * N                                      # R = W
+              + 4 * M * N + 4 * T * N                        # saliency: W and X once each
+              + K * per_base(M, N)
+              + 8 * M * nS_pad                               # gather of the salient columns
+              + Ks * per_base(M, nS_pad))
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            fb.fit(W, X, K, Ks, nS, sweeps)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fb.fit(W, X, K, Ks, nS, sweeps)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out = {"workload": "fit_4096x4096_k2_ks2_s128_sweeps8_t64", "ms_per_fit": round(ms, 3),
+           "algorithmic_bytes": nbytes, "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+           "launches_per_fit": 3 + (K + Ks) * (2 * sweeps + 1) + 1,
+           "note": "fb.fit: saliency, K greedy bases on R = W, gather of the salient columns, Ks bases on them; "
+                   "eager C-ABI calls, median of 5"}
+    if not args.no_cpu:
+        import oracle.fit as ofit
+        t0 = time.perf_counter()
+        ofit.fit(fi.W, fi.X, K, Ks, nS, sweeps)
+        out["cpu_baseline"] = {"ms_per_fit": round((time.perf_counter() - t0) * 1e3, 1), "kind": "oracle",
+                               "cores": len(os.sched_getaffinity(0)), "sample": "one whole fit of the same layer (numpy fp64)"}
     return out
 
 

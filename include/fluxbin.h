@@ -230,6 +230,44 @@ FB_API fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned fl
  * error, else FB_OK. */
 FB_API fb_status fb_device_errors(unsigned int *flags, int clear);
 
+/* ---- The fitter: a dense matrix in, the decomposition's factors out ------
+ * The step before the GEMV.  The FluxBin page (Methodology, 1. Algorithm
+ * innovation: the decoupled row-column binary decomposition and the
+ * Hessian-guided saliency-aware hybrid bases) defines the factors of W_hat
+ * but no fitting procedure; these two calls implement its plainest reading.
+ * Both are asynchronous on `stream`; all pointers are device pointers owned
+ * by the caller; sums are accumulated in fp64 in a fixed order, so results
+ * are reproducible; argument errors return before anything is enqueued.
+ *
+ * fb_fit_saliency: the diagonal-Hessian proxy for choosing the salient
+ * columns.  W [M][ldw] and calibration activations X [T][ldx], fp32
+ * row-major (the first N columns used):
+ *   score[j] = (sum_t X[t][j]^2) * (sum_i W[i][j]^2)          j < N, fp32 out
+ *   s_idx    = the nS columns of largest score (equal scores: the lower
+ *              column first), in ascending order              uint32 [nS] out
+ * 1 <= N <= 65536 (the selection runs in one block: O(N^2 / 1024) compares
+ * per thread), 0 <= nS <= N, ldw, ldx >= N.  s_idx may be NULL when nS = 0.
+ * Returns FB_ERR_INVALID_VALUE / FB_ERR_MISALIGNED (4-byte alignment) for bad
+ * arguments, FB_ERR_CUDA if a launch fails. */
+FB_API fb_status fb_fit_saliency(const float *W, int M, int N, int ldw, const float *X, int T, int ldx, int nS,
+                                 float *score, uint32_t *s_idx, void *stream);
+
+/* fb_fit_base: one greedy base of the decomposition on the residual R
+ * [M][ldr] fp32 (updated in place):
+ *   signs[i][j] = R[i][j] >= 0 ? +1 : -1 (negative zero gives +1)   int8 [M][lds]
+ *   (alpha_r, alpha_c) = the rank-one least-squares fit of |R|, after
+ *     `sweeps` alternating sweeps from alpha_c = 1:
+ *       alpha_r = |R| alpha_c / ||alpha_c||^2, then alpha_c = |R|^T alpha_r /
+ *       ||alpha_r||^2 (a zero norm gives zero scales)     fp32 [M], [N] out
+ *   R[i][j] -= (alpha_r[i] * alpha_c[j]) * signs[i][j]   (fp32, the product
+ *     rounded once, then the update)
+ * Called K times from R = W this yields the global bases; called on the
+ * residual's salient columns (gathered with fb_vcm_gather, zero padding
+ * included) it yields the salient bases.  1 <= sweeps <= 1000, ldr, lds >= N,
+ * M <= 2^24, N <= 2^20.  Errors as fb_fit_saliency. */
+FB_API fb_status fb_fit_base(float *R, int M, int N, int ldr, int sweeps, int8_t *signs, int lds, float *alpha_r,
+                             float *alpha_c, void *stream);
+
 /* Human-readable name of a status code (static string). */
 FB_API const char *fb_status_string(fb_status s);
 

@@ -16,7 +16,7 @@ from __future__ import annotations
 
 import ctypes as C
 import os
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -25,6 +25,7 @@ __all__ = [
     "fb_packed_words", "fb_pack", "fb_pack_bits", "fb_unpack", "fb_vcm_gather",
     "fb_lut_build", "fb_validate_weights", "fb_gemv_workspace_bytes", "fb_gemv",
     "fb_gemv_batched", "fb_status_string", "fb_gemv_launch_plan", "fb_gemv_grouped", "fb_device_errors",
+    "fb_fit_saliency", "fb_fit_base", "fit",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -83,6 +84,8 @@ def lib() -> C.CDLL:
             "fb_gemv_launch_plan": (I, [W, I, C.c_uint, I, P]),
             "fb_gemv_grouped": (I, [P, I, P, I, P, C.c_uint, P]),
             "fb_device_errors": (I, [P, I]),
+            "fb_fit_saliency": (I, [P, I, I, I, P, I, I, I, P, P, P]),
+            "fb_fit_base": (I, [P, I, I, I, I, P, I, P, P, P]),
             "fb_status_string": (C.c_char_p, [I]),
             "fb_abi_version": (I, []),
         }
@@ -305,3 +308,78 @@ def fb_gemv_grouped(Ws, x: torch.Tensor, ys=None, flags: int = 0):
                                  C.cast(yp, C.c_void_p), flags, _stream(x.device)), "fb_gemv_grouped")
     return ys
 
+
+def _f32_rows(t: torch.Tensor, what: str) -> torch.Tensor:
+    if t.dim() != 2 or t.dtype != torch.float32 or t.stride(1) != 1:
+        raise ValueError(f"{what}: a float32 matrix with unit column stride")
+    return t
+
+
+def fb_fit_saliency(W: torch.Tensor, X: torch.Tensor, nS: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Column scores (diagonal-Hessian proxy) and the nS salient columns.
+    W [M, N], X [T, N] fp32 on the GPU -> (score fp32 [N], s_idx int32 [nS],
+    ascending)."""
+    W, X = _f32_rows(W, "W"), _f32_rows(X, "X")
+    M, N = W.shape
+    T = X.shape[0]
+    if X.shape[1] != N:
+        raise ValueError("X must have W's columns")
+    score = torch.empty(N, dtype=torch.float32, device=W.device)
+    s_idx = torch.empty(max(nS, 0), dtype=torch.int32, device=W.device)
+    _check(lib().fb_fit_saliency(W.data_ptr(), M, N, W.stride(0), X.data_ptr(), T, X.stride(0), nS,
+                                 score.data_ptr(), s_idx.data_ptr() if nS > 0 else None, _stream(W.device)),
+           "fb_fit_saliency")
+    return score, s_idx
+
+
+def fb_fit_base(R: torch.Tensor, sweeps: int, signs: Optional[torch.Tensor] = None,
+                alpha_r: Optional[torch.Tensor] = None,
+                alpha_c: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """One greedy base on the residual R [M, N] fp32 (updated in place) ->
+    (signs int8 [M, N], alpha_r fp32 [M], alpha_c fp32 [N]), written into the
+    given outputs when passed (signs: unit column stride; scales contiguous)."""
+    R = _f32_rows(R, "R")
+    M, N = R.shape
+    signs = torch.empty((M, N), dtype=torch.int8, device=R.device) if signs is None else signs
+    ar = torch.empty(M, dtype=torch.float32, device=R.device) if alpha_r is None else alpha_r
+    ac = torch.empty(N, dtype=torch.float32, device=R.device) if alpha_c is None else alpha_c
+    if (signs.shape != (M, N) or signs.dtype != torch.int8 or signs.stride(1) != 1 or ar.shape != (M,)
+            or ac.shape != (N,) or not ar.is_contiguous() or not ac.is_contiguous()):
+        raise ValueError("fb_fit_base: output shapes")
+    _check(lib().fb_fit_base(R.data_ptr(), M, N, R.stride(0), sweeps, signs.data_ptr(), signs.stride(0),
+                             ar.data_ptr(), ac.data_ptr(), _stream(R.device)), "fb_fit_base")
+    return signs, ar, ac
+
+
+def fit(W: torch.Tensor, X: torch.Tensor, K: int, Ks: int, nS: int, sweeps: int) -> dict:
+    """The whole fit on the GPU: K global bases on R = W, then the salient
+    set and Ks bases on the residual's salient columns (gathered by
+    fb_vcm_gather, padded to a multiple of 32 with zero columns).  Returns
+    signs [K, M, N], alpha_r [K, M], alpha_c [K, N], score [N], s_idx [nS],
+    s_signs [Ks, M, nS], s_alpha_r [Ks, M], s_alpha_c [Ks, nS], residual
+    [M, N] (after the global bases) and s_residual [M, nS] (after the salient
+    ones)."""
+    W = _f32_rows(W, "W")
+    M, N = W.shape
+    dev = W.device
+    score, s_idx = fb_fit_saliency(W, X, nS)
+    R = W.clone()
+    signs = torch.empty((K, M, N), dtype=torch.int8, device=dev)
+    ar = torch.empty((K, M), dtype=torch.float32, device=dev)
+    ac = torch.empty((K, N), dtype=torch.float32, device=dev)
+    for k in range(K):
+        fb_fit_base(R, sweeps, signs[k], ar[k], ac[k])
+    nS_pad = (nS + 31) // 32 * 32
+    # the salient bases run over the padded gather (zero columns past nS);
+    # the views below drop the padding
+    s_signs = torch.empty((Ks, M, nS_pad), dtype=torch.int8, device=dev)
+    s_ar = torch.empty((Ks, M), dtype=torch.float32, device=dev)
+    s_ac = torch.empty((Ks, nS_pad), dtype=torch.float32, device=dev)
+    RS = None
+    if nS > 0 and Ks > 0:
+        RS = fb_vcm_gather(R, s_idx, nS_pad)
+        for k in range(Ks):
+            fb_fit_base(RS, sweeps, s_signs[k], s_ar[k], s_ac[k])
+    return {"signs": signs, "alpha_r": ar, "alpha_c": ac, "score": score, "s_idx": s_idx,
+            "s_signs": s_signs[:, :, :nS], "s_alpha_r": s_ar, "s_alpha_c": s_ac[:, :nS], "residual": R,
+            "s_residual": None if RS is None else RS[:, :nS]}

@@ -232,3 +232,24 @@ def test_layout_spec_is_a_bijection():
                     assert len(pos) == 1
                     seen[pos[0]] += 1
         assert seen.max() == 1
+
+
+def test_fit_calls_reject_bad_arguments(L):
+    """The fitter's entry points check every argument on the host and return
+    before any launch (nothing here touches a GPU)."""
+    F, P = FAKE, FAKE + 4
+    sal = L.fb_fit_saliency
+    assert sal(None, 8, 64, 64, F, 4, 64, 3, F, F, None) == INVALID            # no W
+    assert sal(F, 0, 64, 64, F, 4, 64, 3, F, F, None) == INVALID               # M = 0
+    assert sal(F, 8, 65537, 65537, F, 4, 65537, 3, F, F, None) == INVALID      # N past the one-block selection
+    assert sal(F, 8, 64, 63, F, 4, 64, 3, F, F, None) == INVALID               # ldw < N
+    assert sal(F, 8, 64, 64, F, 4, 64, 65, F, F, None) == INVALID              # nS > N
+    assert sal(F, 8, 64, 64, F, 4, 64, 3, F, None, None) == INVALID            # nS > 0 without s_idx
+    assert sal(F + 1, 8, 64, 64, F, 4, 64, 3, F, F, None) == MISALIGNED
+    base = L.fb_fit_base
+    assert base(F, 8, 64, 64, 0, F, 64, F, F, None) == INVALID                 # no sweep
+    assert base(F, 8, 64, 64, 1001, F, 64, F, F, None) == INVALID
+    assert base(F, 8, 64, 32, 2, F, 64, F, F, None) == INVALID                 # ldr < N
+    assert base(F, 8, 64, 64, 2, F, 63, F, F, None) == INVALID                 # lds < N
+    assert base(None, 8, 64, 64, 2, F, 64, F, F, None) == INVALID
+    assert base(F, 8, 64, 64, 2, F, 64, P + 1, F, None) == MISALIGNED
