@@ -28,6 +28,8 @@ namespace {
 constexpr int kFitMaxN = 65536;        // salient selection runs in one block, a bit per column
 constexpr int kFitMaxSweeps = 1000;
 constexpr int kSelectThreads = 1024;
+constexpr int kColUnroll = 16;   // rows a lane loads before adding them (memory requests in flight)
+constexpr int kRowUnroll = 8;    // columns a lane loads before adding them
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -62,11 +64,20 @@ __global__ void __launch_bounds__(256) colsumsq_kernel(const float *A, int rows,
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int j = blockIdx.x * 32 + lane;
     double s = 0.0;
-    if (j < cols)
-        for (int i = w; i < rows; i += 8) {
+    if (j < cols) {
+        int i = w;
+        for (; i + 8 * (kColUnroll - 1) < rows; i += 8 * kColUnroll) {   // same order, loads issued first
+            float v[kColUnroll];
+#pragma unroll
+            for (int u = 0; u < kColUnroll; ++u) v[u] = A[(size_t)(i + 8 * u) * ld + j];
+#pragma unroll
+            for (int u = 0; u < kColUnroll; ++u) s = fma((double)v[u], (double)v[u], s);
+        }
+        for (; i < rows; i += 8) {
             const double v = A[(size_t)i * ld + j];
             s = fma(v, v, s);
         }
+    }
     part[w][lane] = s;
     __syncthreads();
     if (w == 0 && j < cols) {
@@ -138,7 +149,18 @@ __global__ void __launch_bounds__(256) fit_rows_kernel(const float *R, int M, in
     if (i >= M) return;
     const float *row = R + (size_t)i * ld;
     double s = 0.0;
-    for (int j = lane; j < N; j += 32) s = fma((double)fabsf(row[j]), ones ? 1.0 : (double)ac[j], s);
+    int j = lane;
+    for (; j + 32 * (kRowUnroll - 1) < N; j += 32 * kRowUnroll) {   // same order, loads issued first
+        float v[kRowUnroll], c[kRowUnroll];
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) {
+            v[u] = row[j + 32 * u];
+            c[u] = ones ? 1.0f : ac[j + 32 * u];
+        }
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) s = fma((double)fabsf(v[u]), (double)c[u], s);
+    }
+    for (; j < N; j += 32) s = fma((double)fabsf(row[j]), ones ? 1.0 : (double)ac[j], s);
     s = warp_sum(s);
     if (lane == 0) ar[i] = nc > 0.0 ? (float)(s / nc) : 0.0f;
 }
@@ -154,8 +176,20 @@ __global__ void __launch_bounds__(256) fit_cols_kernel(const float *R, int M, in
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int j = blockIdx.x * 32 + lane;
     double s = 0.0;
-    if (j < N)
-        for (int i = w; i < M; i += 8) s = fma((double)fabsf(R[(size_t)i * ld + j]), (double)ar[i], s);
+    if (j < N) {
+        int i = w;
+        for (; i + 8 * (kColUnroll - 1) < M; i += 8 * kColUnroll) {   // same order, loads issued first
+            float v[kColUnroll], a[kColUnroll];
+#pragma unroll
+            for (int u = 0; u < kColUnroll; ++u) {
+                v[u] = R[(size_t)(i + 8 * u) * ld + j];
+                a[u] = ar[i + 8 * u];
+            }
+#pragma unroll
+            for (int u = 0; u < kColUnroll; ++u) s = fma((double)fabsf(v[u]), (double)a[u], s);
+        }
+        for (; i < M; i += 8) s = fma((double)fabsf(R[(size_t)i * ld + j]), (double)ar[i], s);
+    }
     part[w][lane] = s;
     __syncthreads();
     if (w == 0 && j < N) {
