@@ -19,7 +19,8 @@ g = 8 variant on the same weights, the 7B-shaped decode step (224 GEMVs), the
 roofline of the GEMV kernel against the measured HBM peak, every workload at
 its own shape, a dense fp16 comparator with energy per call, e2e through the
 public API with pinned host buffers copied in and out every step (graph-replayed
-and eager calls), and the fp64 CPU oracle as baseline.
+and eager calls), the fitter (a whole 4096 x 4096 fit from a dense layer), and
+the fp64 CPU oracle as baseline.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
