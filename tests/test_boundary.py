@@ -253,3 +253,17 @@ def test_fit_calls_reject_bad_arguments(L):
     assert base(F, 8, 64, 64, 2, F, 63, F, F, None) == INVALID                 # lds < N
     assert base(None, 8, 64, 64, 2, F, 64, F, F, None) == INVALID
     assert base(F, 8, 64, 64, 2, F, 64, P + 1, F, None) == MISALIGNED
+
+
+def test_fit_binding_checks_shapes_before_calling():
+    """The Python fitter calls refuse wrong dtypes and shapes before reaching
+    the library (CPU tensors suffice: nothing is launched)."""
+    import torch
+    with pytest.raises(ValueError):
+        fb.fb_fit_base(torch.zeros((3, 4), dtype=torch.float64), 2)
+    with pytest.raises(ValueError):
+        fb.fb_fit_base(torch.zeros((3, 4)).t(), 2)                      # columns not contiguous
+    with pytest.raises(ValueError):
+        fb.fb_fit_saliency(torch.zeros((3, 4)), torch.zeros((2, 5)), 1)   # X has other columns
+    with pytest.raises(ValueError):
+        fb.fb_fit_base(torch.zeros((3, 4)), 2, signs=torch.zeros((3, 4), dtype=torch.int32))
