@@ -105,3 +105,23 @@ def test_fit_saliency_writes_only_its_outputs():
     assert bool((score[N:] == SENT_F).all()) and bool((s_idx[nS:] == SENT_I32).all())
     sc, si = fb.fb_fit_saliency(Wt, Xt, nS)
     assert torch.equal(score[:N], sc) and torch.equal(s_idx[:nS], si)
+
+
+def test_lut_build_and_unpack_write_only_their_outputs():
+    K, M, N, g = 2, 45, 96, 4
+    rng = np.random.default_rng(57)
+    x = torch.from_numpy(rng.normal(size=N).astype(np.float32)).to(DEV)
+    ac = torch.from_numpy(rng.uniform(0.5, 2.0, size=(K, N)).astype(np.float32)).to(DEV)
+    n = K * (N // g) * (1 << g)
+    lut = torch.full((n + 32,), SENT_F, device=DEV)
+    assert fb.lib().fb_lut_build(x.data_ptr(), 0, ac.data_ptr(), K, N, g, lut.data_ptr(), _stream()) == 0
+    torch.cuda.synchronize()
+    assert bool((lut[n:] == SENT_F).all())
+    assert torch.equal(lut[:n], fb.fb_lut_build(x, ac, K, g).reshape(-1))
+    signs = torch.from_numpy(np.where(rng.random((K, M, N)) < 0.5, 1, -1).astype(np.int8)).to(DEV)
+    planes = fb.fb_pack(signs)
+    out = torch.full((K * M * N + 64,), SENT_I8, dtype=torch.int8, device=DEV)
+    assert fb.lib().fb_unpack(planes.data_ptr(), K, M, N, out.data_ptr(), _stream()) == 0
+    torch.cuda.synchronize()
+    assert bool((out[K * M * N:] == SENT_I8).all())
+    assert torch.equal(out[: K * M * N].view(K, M, N), signs)
