@@ -56,9 +56,10 @@ def test_hand_worked_example():
     x = np.array(ex["x"], np.float64)
     W = oracle.dequant(w)
     assert np.array_equal(W, np.array(ex["expected"]["W"]))
-    y, d, _ = oracle.gemv(w, x)
+    y, d, e = oracle.gemv(w, x)
     assert np.array_equal(y[0], ex["expected"]["y"])
     assert np.array_equal(d[0], ex["expected"]["d"])
+    assert np.array_equal(e[0], ex["expected"]["e"])
     for g in (1, 2, 4, 8):
         assert np.array_equal(oracle.gemv_lut(w, g, x)[0], ex["expected"]["y"])
     T = oracle.lut_tables(x, np.array(ex["alpha_c"], np.float32), 2, 4)
