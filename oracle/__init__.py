@@ -50,6 +50,8 @@ def lib():
         L = C.CDLL(path)
         P = C.c_void_p
         L.oracle_num_threads.restype = C.c_int
+        L.oracle_set_num_threads.argtypes = [C.c_int]
+        L.oracle_set_num_threads.restype = None
         L.oracle_x_to_f64.argtypes = [C.c_int, P, C.c_int64, P]
         L.oracle_dequant_rows.argtypes = [C.POINTER(_Weights), C.c_int64, P, P]
         L.oracle_gemv.argtypes = [C.POINTER(_Weights), P, C.c_int, C.c_int64, P, P, P, P]
@@ -65,6 +67,12 @@ def lib():
 
 def num_threads() -> int:
     return lib().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the oracle's parallel loops use (timing aid; results do not
+    depend on it)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def _ptr(a: Optional[np.ndarray]):

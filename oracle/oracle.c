@@ -59,6 +59,13 @@ enum { ORACLE_OK = 0, ORACLE_EINVAL = -1, ORACLE_ENOMEM = -2 };
 
 int oracle_num_threads(void) { return omp_get_max_threads(); }
 
+/* Threads the parallel loops use from now on (n >= 1); for timing the oracle
+ * on one core beside all cores.  Changes no arithmetic: rows are independent
+ * and each row's sums run in the order written whatever the thread count. */
+void oracle_set_num_threads(int n) {
+    if (n >= 1) omp_set_num_threads(n);
+}
+
 /* ---- activations: stored dtype -> double, exactly ------------------------ */
 
 static double f16_to_f64(uint16_t h) {
