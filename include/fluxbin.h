@@ -125,12 +125,14 @@ FB_API fb_status fb_lut_build(const void *x, fb_dtype t, const float *alpha_c, i
 /* Weights of one M x N linear layer.  Host struct; every pointer in it is a
  * device pointer owned by the caller. */
 typedef struct fb_weights {
-    int M, N, K, g;              /* g: LUT group width (1, 2, 4 or 8).  fb_gemv
-                                    looks up one weight byte (8 columns) per
-                                    table access for every g: each byte-table
-                                    entry is the sum of the byte's 8/g
-                                    g-column LUT entries, added pairwise, so g
-                                    fixes the grouping of the fp32 sums */
+    int M, N, K, g;              /* g: LUT group width (1, 2, 4 or 8), checked
+                                    but NOT used by the GEMV calls: they always
+                                    look up one weight byte (8 columns) per
+                                    table access in 256-entry tables, each
+                                    entry formed as the sum of the two
+                                    4-column tables of its nibbles, so every
+                                    g gives the same result bits.  g is the
+                                    table width of fb_lut_build */
     const uint32_t *planes;      /* fb_pack(K, M, N) output, 16-byte aligned */
     const float *alpha_r;        /* [K][M] row scales */
     const float *alpha_c;        /* [K][N] column scales, or NULL for all ones */
@@ -207,6 +209,23 @@ FB_API fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtype t,
  * matrices together need more than 65535 row blocks. */
 FB_API fb_status fb_gemv_grouped(const fb_weights *const *W, int n, const void *x, fb_dtype t, float *const *y,
                                  unsigned flags, void *stream);
+
+/* fb_gemv_group_scales: y = W_hat x (batch 1) for the group-wise row-scale
+ * format, one row scale per group of G consecutive input columns:
+ *   W_hat[i][j] = sum_k alpha_r[k][j / G][i] * alpha_c[k][j] * B^(k)[i][j]
+ *                 + the salient term, whose row scales stay per row.
+ * The FluxBin page names this variant only through its "2b-s16-g128"
+ * setting (Experimental results, the accuracy paragraph) and does not define
+ * it; G = 128 is that setting's reading.  W is an ordinary fb_weights except
+ * that W->alpha_r holds K * (N / G) row-scale vectors of M floats, laid out
+ * [K][N/G][M] (group g of base k at alpha_r + (k * N/G + g) * M).  G = 128,
+ * N, or a multiple of 256 dividing N, else FB_ERR_INVALID_VALUE; G = N is the
+ * ordinary format (the same result bits as fb_gemv).  x, t, y, flags and the result's properties (fp32 sums,
+ * deterministic, tolerance) as for fb_gemv.  With G = 128 every 256-column
+ * panel is looked up once per half (the other half's columns contributing
+ * exact zeros), so a call costs about twice the table work of fb_gemv. */
+FB_API fb_status fb_gemv_group_scales(const fb_weights *W, int G, const void *x, fb_dtype t, float *y,
+                                      unsigned flags, void *stream);
 
 /* fb_gemv_launch_plan: diagnostic, host only.  The launch shape fb_gemv /
  * fb_gemv_batched use for W at this batch size and these flags (calls flagged

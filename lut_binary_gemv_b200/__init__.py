@@ -25,7 +25,7 @@ __all__ = [
     "fb_packed_words", "fb_pack", "fb_pack_bits", "fb_unpack", "fb_vcm_gather",
     "fb_lut_build", "fb_validate_weights", "fb_gemv_workspace_bytes", "fb_gemv",
     "fb_gemv_batched", "fb_status_string", "fb_gemv_launch_plan", "fb_gemv_grouped", "fb_device_errors",
-    "fb_fit_saliency", "fb_fit_base", "fit",
+    "fb_fit_saliency", "fb_fit_base", "fit", "fb_gemv_group_scales",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -83,6 +83,7 @@ def lib() -> C.CDLL:
             "fb_gemv_batched": (I, [W, P, I, I, I, P, I, P, S, C.c_uint, P]),
             "fb_gemv_launch_plan": (I, [W, I, C.c_uint, I, P]),
             "fb_gemv_grouped": (I, [P, I, P, I, P, C.c_uint, P]),
+            "fb_gemv_group_scales": (I, [W, I, P, I, P, C.c_uint, P]),
             "fb_device_errors": (I, [P, I]),
             "fb_fit_saliency": (I, [P, I, I, I, P, I, I, I, P, P, P]),
             "fb_fit_base": (I, [P, I, I, I, I, P, I, P, P, P]),
@@ -307,6 +308,26 @@ def fb_gemv_grouped(Ws, x: torch.Tensor, ys=None, flags: int = 0):
     _check(lib().fb_gemv_grouped(C.cast(wp, C.c_void_p), n, x.data_ptr(), _DTYPES[x.dtype],
                                  C.cast(yp, C.c_void_p), flags, _stream(x.device)), "fb_gemv_grouped")
     return ys
+
+
+def fb_gemv_group_scales(W: Weights, G: int, x: torch.Tensor, alpha_r_groups: torch.Tensor,
+                         y: Optional[torch.Tensor] = None, flags: int = 0) -> torch.Tensor:
+    """y = W_hat x with one row scale per group of G input columns:
+    alpha_r_groups fp32 [K, N/G, M] (replacing W.alpha_r); W's other tensors
+    as for fb_gemv."""
+    if x.stride(-1) != 1:
+        x = x.contiguous()
+    if G <= 0 or W.N % G:
+        raise ValueError("G must be a positive divisor of N")
+    if (alpha_r_groups.dtype != torch.float32 or not alpha_r_groups.is_contiguous()
+            or alpha_r_groups.numel() != W.K * (W.N // G) * W.M):
+        raise ValueError("alpha_r_groups: contiguous float32 [K, N/G, M]")
+    y = torch.empty(W.M, dtype=torch.float32, device=x.device) if y is None else y
+    st = FbWeightsStruct.from_buffer_copy(W.struct)
+    st.alpha_r = alpha_r_groups.data_ptr()
+    _check(lib().fb_gemv_group_scales(C.byref(st), G, x.data_ptr(), _DTYPES[x.dtype], y.data_ptr(), flags,
+                                      _stream(x.device)), "fb_gemv_group_scales")
+    return y
 
 
 def _f32_rows(t: torch.Tensor, what: str) -> torch.Tensor:

@@ -158,7 +158,7 @@ def test_other_entry_points_reject_bad_arguments(L):
     (4096, 11008, 2, 4, 330, 2), (8192, 8192, 3, 8, 410, 2), (28672, 8192, 3, 8, 410, 2),
     (8192, 28672, 3, 8, 1434, 2), (131077, 64, 1, 2, 0, 0), (100, 800, 4, 1, 800, 4),
 ])
-@pytest.mark.parametrize("batch", [1, 16])
+@pytest.mark.parametrize("batch", [1, 16, 64])
 @pytest.mark.parametrize("flags", [0, 1, 3])
 def test_launch_plan_covers_the_matrix(L, shape, batch, flags):
     M, N, K, g, nS, Ks = shape
@@ -168,23 +168,46 @@ def test_launch_plan_covers_the_matrix(L, shape, batch, flags):
     P = lambda n: -(-n // 256)
     V = P(N) * K + (P(-(-nS // 32) * 32) * Ks if nS else 0)
     assert plan["V"] == V
-    assert 1 <= plan["C"] <= min(8, V)
+    assert 1 <= plan["C"] <= min(16, V)
     assert plan["RB"] * plan["cpb"] >= nchunks > (plan["RB"] - 1) * plan["cpb"]
-    assert plan["warps"] in (8, 16)
+    assert plan["cpb"] <= 32
+    assert plan["warps"] == (8 if batch == 1 else 16)
     assert 0 < plan["smem"] <= 225 * 1024
 
 
+@pytest.mark.parametrize("M", [1, 32, 4096, 1 << 24])
+@pytest.mark.parametrize("N", [32, 4096, 1 << 20])
+@pytest.mark.parametrize("K,nS,Ks", [(1, 0, 1), (4, 0, 1), (4, -1, 4)])
+@pytest.mark.parametrize("batch", [1, 2, 64])
+@pytest.mark.parametrize("flags", [0, 1, 3])
+def test_launch_plan_fits_at_the_abi_corners(L, M, N, K, nS, Ks, batch, flags):
+    """Every plan the ABI's extreme sizes can ask for fits one CTA's shared
+    memory, stays within the grid's row-block limit and covers the matrix
+    (nS = -1: every column salient)."""
+    nS = N if nS < 0 else nS
+    s = fake_weights(M=M, N=N, K=K, g=4, nS=nS, Ks=Ks)
+    plan = fb.fb_gemv_launch_plan(s, batch, flags, 148)
+    nchunks = -(-M // 32)
+    assert 0 < plan["smem"] <= 225 * 1024
+    assert 1 <= plan["C"] <= min(16, plan["V"])
+    assert plan["RB"] <= 65535
+    assert plan["RB"] * plan["cpb"] >= nchunks > (plan["RB"] - 1) * plan["cpb"]
+
+
 def test_launch_plan_shapes_by_call_kind(L):
-    """Calls flagged independent get the 16-warp CTA (row blocks of up to 32
-    chunks); dependent calls the 8-warp CTA (up to 16 chunks, a whole number
-    of chunks per warp when the matrix has enough)."""
+    """Batch-1 calls get the 8-warp streaming CTA (two per SM) with rows in
+    whole chunks per warp; calls flagged independent take row blocks of up to
+    32 chunks; dependent calls one wave over the GPU.  Batched calls get the
+    16-warp batched CTA."""
     for M, N, K, g, nS, Ks in ((4096, 4096, 2, 4, 128, 2), (11008, 4096, 2, 4, 123, 2), (8192, 8192, 3, 8, 410, 2)):
         s = fake_weights(M=M, N=N, K=K, g=g, nS=nS, Ks=Ks)
         ind = fb.fb_gemv_launch_plan(s, 1, 3, 148)
         dep = fb.fb_gemv_launch_plan(s, 1, 1, 148)
-        assert ind["warps"] == 16 and ind["cpb"] <= 32
-        assert dep["warps"] == 8 and dep["cpb"] <= 16 and dep["cpb"] % 8 == 0
+        bat = fb.fb_gemv_launch_plan(s, 16, 1, 148)
+        assert ind["warps"] == 8 and ind["cpb"] <= 32
+        assert dep["warps"] == 8 and dep["cpb"] <= 32 and dep["cpb"] % 8 == 0
         assert dep["C"] * dep["RB"] <= 2 * 148        # one wave at two CTAs per SM
+        assert bat["warps"] == 16 and bat["C"] * bat["RB"] <= 148
 
 
 def test_launch_plan_rejects_bad_arguments(L):

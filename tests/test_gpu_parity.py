@@ -405,6 +405,16 @@ def test_workload_70b(shape_index, batch):
         check(pi, run_gpu(pi), sample_rows(pi.M, 64, 10 + shape_index))
 
 
+@pytest.mark.parametrize("batch", [1, 16])
+def test_workload_70b_every_row(batch):
+    """The 28672 x 8192 layer (K = 3, g = 8, 5% salient) checked on every
+    row of every token, in both launch plans of batch-1 calls."""
+    p = wl.layer70b(1, batch)
+    check(p, run_gpu(p))
+    if batch == 1:
+        check(p, run_gpu(p, flags=fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT))
+
+
 @pytest.mark.gpu
 def test_device_error_flags_stay_clear():
     # every bounded wait for a weight copy in the runs above ended in time
