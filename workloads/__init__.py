@@ -164,6 +164,15 @@ def _x(rng: np.random.Generator, batch: int, n: int, dtype: str,
     raise ValueError(dtype)
 
 
+def group_row_scales(K: int, M: int, ngroups: int, *, seed, alpha_dist: str = "small",
+                     integer_mode: bool = False) -> np.ndarray:
+    """Row scales of the group-wise format, one per (base, row, group of
+    input columns): float32 [K][M][ngroups], drawn like the per-row scales
+    (same distributions, same integer-mode values) from their own seed."""
+    rng = np.random.default_rng(seed)
+    return _alpha(rng, (K, M, ngroups), alpha_dist, integer_mode, row_scale=True)
+
+
 def make_problem(M: int, N: int, K: int, *, g: int = 4, nS: int = 0, Ks: int = 2,
                  batch: int = 1, x_dtype: str = "f32", alpha_dist: str = "small",
                  seed=0, integer_mode: bool = False, ternary: bool = False,
