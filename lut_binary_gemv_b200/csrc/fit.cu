@@ -17,10 +17,13 @@
 // Every sum is accumulated in fp64 in a fixed order (results do not depend
 // on scheduling); scales and the residual are stored as fp32.  All of it is
 // bandwidth-bound streaming over R, with no tensor-core work.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "fb_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace fb {
 namespace {
@@ -55,36 +58,69 @@ __device__ double block_norm2(const float *v, int n, double *red) {
     return t;
 }
 
-// out[j] = sum_i A[i][j]^2 (multiply = 0), or out[j] *= that sum (multiply =
-// 1).  A block of 8 warps covers 32 columns: warp w sums rows w, w + 8, ...,
-// lane = column; the 8 partial sums are added in warp order.
-__global__ void __launch_bounds__(256) colsumsq_kernel(const float *A, int rows, int cols, int ld, float *out,
-                                                        int multiply) {
+// Column passes split the rows over a cluster of kColSplit CTAs: CTA r of
+// the cluster sums row slice r of its 32 columns (8 warps, warp w taking rows
+// w, w + 8, ... of the slice, the 8 partials added in warp order) and sends
+// its 32 sums to rank 0's shared memory; rank 0 adds the kColSplit slices in
+// rank order.  A fixed order throughout, so results do not depend on
+// scheduling, and no scratch memory.
+constexpr int kColSplit = 8;
+
+// Sum over row slice `rank` of f(A[i][j]) * w(i) for this lane's column j, in
+// the order described above; returns this CTA's 32 partials' rank-0 total in
+// lane order on rank 0 (other ranks return 0).
+template <typename Term>
+__device__ double cluster_column_sum(int rows, int j, bool valid, Term term) {
     __shared__ double part[8][32];
+    __shared__ double inbox[kColSplit][32];
+    cg::cluster_group cl = cg::this_cluster();
+    const int rank = (int)cl.block_rank();
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int j = blockIdx.x * 32 + lane;
+    const int rs = (rows + kColSplit - 1) / kColSplit, i0 = rank * rs, i1 = min(rows, i0 + rs);
     double s = 0.0;
-    if (j < cols) {
-        int i = w;
-        for (; i + 8 * (kColUnroll - 1) < rows; i += 8 * kColUnroll) {   // same order, loads issued first
-            float v[kColUnroll];
+    if (valid) {
+        int i = i0 + w;
+        for (; i + 8 * (kColUnroll - 1) < i1; i += 8 * kColUnroll) {   // same order, loads issued first
+            double v[kColUnroll];
 #pragma unroll
-            for (int u = 0; u < kColUnroll; ++u) v[u] = A[(size_t)(i + 8 * u) * ld + j];
+            for (int u = 0; u < kColUnroll; ++u) v[u] = term.load(i + 8 * u, j);
 #pragma unroll
-            for (int u = 0; u < kColUnroll; ++u) s = fma((double)v[u], (double)v[u], s);
+            for (int u = 0; u < kColUnroll; ++u) s = term.add(s, v[u], i + 8 * u);
         }
-        for (; i < rows; i += 8) {
-            const double v = A[(size_t)i * ld + j];
-            s = fma(v, v, s);
-        }
+        for (; i < i1; i += 8) s = term.add(s, term.load(i, j), i);
     }
     part[w][lane] = s;
     __syncthreads();
-    if (w == 0 && j < cols) {
+    if (w == 0) {
         double t = part[0][lane];
         for (int q = 1; q < 8; ++q) t += part[q][lane];
-        out[j] = multiply ? (float)((double)out[j] * t) : (float)t;
+        cl.map_shared_rank(&inbox[0][0], 0)[rank * 32 + lane] = t;
     }
+    cl.sync();
+    double total = 0.0;
+    if (rank == 0 && w == 0) {
+        total = inbox[0][lane];
+        for (int q = 1; q < kColSplit; ++q) total += inbox[q][lane];
+    }
+    return total;
+}
+
+struct SumSquares {
+    const float *A;
+    int ld;
+    __device__ double load(int i, int j) const { return (double)A[(size_t)i * ld + j]; }
+    __device__ double add(double s, double v, int) const { return fma(v, v, s); }
+};
+
+// out[j] = sum_i A[i][j]^2 (multiply = 0), or out[j] *= that sum (multiply =
+// 1).  grid.x = kColSplit * (column blocks of 32).
+__global__ void __cluster_dims__(kColSplit, 1, 1) __launch_bounds__(256)
+    colsumsq_kernel(const float *A, int rows, int cols, int ld, float *out, int multiply) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int j = (int)(blockIdx.x / kColSplit) * 32 + lane;
+    const double t = cluster_column_sum(rows, j, j < cols, SumSquares{A, ld});
+    if (cg::this_cluster().block_rank() == 0 && w == 0 && j < cols)
+        out[j] = multiply ? (float)((double)out[j] * t) : (float)t;
 }
 
 // Order-preserving key of a float: a larger float has a larger key, and every
@@ -165,38 +201,25 @@ __global__ void __launch_bounds__(256) fit_rows_kernel(const float *R, int M, in
     if (lane == 0) ar[i] = nc > 0.0 ? (float)(s / nc) : 0.0f;
 }
 
-// alpha_c[j] = sum_i |R[i][j]| alpha_r[i] / ||alpha_r||^2.  A block of 8 warps
-// covers 32 columns: warp w takes rows w, w + 8, ...; partials added in warp
-// order.
-__global__ void __launch_bounds__(256) fit_cols_kernel(const float *R, int M, int N, int ld, const float *ar,
-                                                        float *ac) {
+struct AbsTimesRowScale {
+    const float *R;
+    int ld;
+    const float *ar;
+    __device__ double load(int i, int j) const { return (double)fabsf(R[(size_t)i * ld + j]); }
+    __device__ double add(double s, double v, int i) const { return fma(v, (double)ar[i], s); }
+};
+
+// alpha_c[j] = sum_i |R[i][j]| alpha_r[i] / ||alpha_r||^2, the rows split over
+// the cluster as above; rank 0 also forms ||alpha_r||^2 (block_norm2 order).
+__global__ void __cluster_dims__(kColSplit, 1, 1) __launch_bounds__(256)
+    fit_cols_kernel(const float *R, int M, int N, int ld, const float *ar, float *ac) {
     __shared__ double red[8];
-    __shared__ double part[8][32];
-    const double nr = block_norm2(ar, M, red);
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int j = blockIdx.x * 32 + lane;
-    double s = 0.0;
-    if (j < N) {
-        int i = w;
-        for (; i + 8 * (kColUnroll - 1) < M; i += 8 * kColUnroll) {   // same order, loads issued first
-            float v[kColUnroll], a[kColUnroll];
-#pragma unroll
-            for (int u = 0; u < kColUnroll; ++u) {
-                v[u] = R[(size_t)(i + 8 * u) * ld + j];
-                a[u] = ar[i + 8 * u];
-            }
-#pragma unroll
-            for (int u = 0; u < kColUnroll; ++u) s = fma((double)fabsf(v[u]), (double)a[u], s);
-        }
-        for (; i < M; i += 8) s = fma((double)fabsf(R[(size_t)i * ld + j]), (double)ar[i], s);
-    }
-    part[w][lane] = s;
-    __syncthreads();
-    if (w == 0 && j < N) {
-        double t = part[0][lane];
-        for (int q = 1; q < 8; ++q) t += part[q][lane];
-        ac[j] = nr > 0.0 ? (float)(t / nr) : 0.0f;
-    }
+    const int j = (int)(blockIdx.x / kColSplit) * 32 + lane;
+    const double t = cluster_column_sum(M, j, j < N, AbsTimesRowScale{R, ld, ar});
+    if (cg::this_cluster().block_rank() != 0) return;
+    const double nr = block_norm2(ar, M, red);
+    if (w == 0 && j < N) ac[j] = nr > 0.0 ? (float)(t / nr) : 0.0f;
 }
 
 // signs = sign(R) (R >= 0 gives +1, -0 included); R -= (alpha_r[i] alpha_c[j])
@@ -229,7 +252,7 @@ extern "C" fb_status fb_fit_saliency(const float *W, int M, int N, int ldw, cons
     if (!aligned(W, 4) || !aligned(X, 4) || !aligned(score, 4) || (s_idx && !aligned(s_idx, 4)))
         return FB_ERR_MISALIGNED;
     cudaStream_t s = as_stream(stream);
-    const dim3 grid(ceil_div(N, 32)), block(256);
+    const dim3 grid(ceil_div(N, 32) * kColSplit), block(256);
     cudaError_t e = launch(colsumsq_kernel, grid, block, 0, s, false, W, M, N, ldw, score, 0);
     if (e == cudaSuccess) e = launch(colsumsq_kernel, grid, block, 0, s, false, X, T, N, ldx, score, 1);
     if (e == cudaSuccess && nS > 0) {
@@ -246,7 +269,7 @@ extern "C" fb_status fb_fit_base(float *R, int M, int N, int ldr, int sweeps, in
         return FB_ERR_INVALID_VALUE;
     if (!aligned(R, 4) || !aligned(alpha_r, 4) || !aligned(alpha_c, 4)) return FB_ERR_MISALIGNED;
     cudaStream_t s = as_stream(stream);
-    const dim3 block(256), rows_grid(ceil_div(M, 8)), cols_grid(ceil_div(N, 32));
+    const dim3 block(256), rows_grid(ceil_div(M, 8)), cols_grid(ceil_div(N, 32) * kColSplit);
     cudaError_t e = cudaSuccess;
     for (int it = 0; it < sweeps && e == cudaSuccess; ++it) {
         e = launch(fit_rows_kernel, rows_grid, block, 0, s, false, (const float *)R, M, N, ldr,
