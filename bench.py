@@ -44,6 +44,7 @@ METRIC = "GEMV µs & achieved HBM GB/s (% peak) at 4096×4096 K=2; 7B-shaped ste
 WEIGHT_SETS = 64
 PASSES_PER_STEP = 16
 FALLBACK_HBM_GBS = 6650.0
+SM_MAX_GHZ = 1.965   # clocks.max.sm of this machine's B200s
 
 
 def parse():
@@ -188,12 +189,14 @@ def workload_config():
 
 # --------------------------------------------------------------------------
 def cpu_baseline(seconds):
-    """The fp64 oracle (dense dequantisation + fp64 dot) on this host's cores."""
+    """The fp64 oracle (dense dequantisation + fp64 dot) on this host's cores:
+    all cores (OpenMP over rows), and one core on a bounded row sample."""
     import oracle
     import workloads as wl
     p = wl.layer4096()
     w = oracle.OracleWeights.from_problem(p)
     x = oracle.x_to_f64(p.x, p.x_dtype)
+    cores = oracle.num_threads()
     oracle.gemv(w, x)                        # warm (page in, thread pool)
     n, t0 = 0, time.perf_counter()
     while True:
@@ -203,9 +206,28 @@ def cpu_baseline(seconds):
         if dt >= seconds:
             break
     per = dt / n
-    return {"value": round(p.algorithmic_bytes() / per / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+    # one core: a bounded sample of rows (about a third of the time budget)
+    oracle.set_num_threads(1)
+    try:
+        rows = 512
+        sel = np.arange(rows)
+        oracle.gemv(w, x, sel)
+        n1, t1 = 0, time.perf_counter()
+        while True:
+            oracle.gemv(w, x, sel)
+            n1 += 1
+            dt1 = time.perf_counter() - t1
+            if dt1 >= seconds / 3:
+                break
+        per1 = dt1 / n1 * (p.M / rows)       # scaled to a whole GEMV
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": round(p.algorithmic_bytes() / per / 1e9, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle", "sample": f"{n} full 4096x4096 K=2 GEMVs (all rows) of the same workload, "
-            f"{per * 1e3:.1f} ms each", "ms_per_gemv": round(per * 1e3, 3)}
+            f"{per * 1e3:.1f} ms each", "ms_per_gemv": round(per * 1e3, 3),
+            "single_core": {"value": round(p.algorithmic_bytes() / per1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                            "ms_per_gemv": round(per1 * 1e3, 3),
+                            "sample": f"{n1} passes over rows 0..{rows - 1} of the same GEMV, scaled to 4096 rows"}}
 
 
 def run_reference(args):
@@ -410,8 +432,9 @@ def run_ours(args):
         step7b = bench_7b(args, device, stream, world, peak)
     configs = None if args.no_configs else bench_configs(args, device, stream, world, peak)
     ours_energy = round(clocks["power_w_mean"] * us_per_gemv, 2) if clocks and clocks.get("power_w_mean") else None
-    fp16 = None if args.no_configs else bench_fp16_dense(args, device, stream, world, gpu_id, us_per_gemv, ours_energy)
+    fp16 = None if args.no_configs else bench_vs_fp16(args, device, stream, world, gpu_id)
     fitter = None if args.no_configs else bench_fit(args, device, stream, peak)
+    group_scales = None if args.no_configs else bench_group_scales(args, device, stream, world, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -436,6 +459,7 @@ def run_ours(args):
         "energy_uj_per_gemv": ours_energy,
         "fp16_dense_comparator": fp16,
         "fitter": fitter,
+        "group_scales": group_scales,
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 4),
                 "note": (f"per step: pinned host x ({n_e2e} x 4096 fp16) copied in, {n_e2e} fb_gemv calls "
@@ -557,8 +581,16 @@ def bench_configs(args, device, stream, world, peak):
             xb = {"f32": 4, "f16": 2, "bf16": 2}[p0.x_dtype]
             nbytes = per_set + B * (p0.N * xb + 4 * p0.M)
             gbs = nbytes / (us * 1e-6) / 1e9
-            res[f"batch{B}"] = {"us_per_call": round(us, 3), "us_per_token": round(us / B, 3), "gbs": round(gbs, 1),
-                                "frac": round(gbs / peak, 4), "weight_sets": len(Ws), "fits_l2": per_set * len(Ws) < l2}
+            r = {"us_per_call": round(us, 3), "us_per_token": round(us / B, 3), "gbs": round(gbs, 1),
+                 "frac": round(gbs / peak, 4), "weight_sets": len(Ws), "fits_l2": per_set * len(Ws) < l2}
+            if B > 1:
+                # shared-memory roof: every weight byte is one 4-byte table
+                # lookup per token; 148 SMs x 128 B per clock at the top clock
+                wbytes = p0.K * p0.M * p0.N // 8 + (p0.Ks * p0.M * p0.nS_pad // 8 if p0.nS else 0)
+                roof_us = B * wbytes * 4 / (148 * 128 * SM_MAX_GHZ * 1e9) * 1e6
+                r["smem_roof"] = {"us": round(roof_us, 3), "frac": round(roof_us / us, 4),
+                                  "basis": "B x weight bytes x 4 B lookups / (148 SMs x 128 B/clk x 1.965 GHz)"}
+            res[f"batch{B}"] = r
             del g, Ys
         out[name] = res if len(batches) > 1 else res["batch1"]
         del Ws, Xs
@@ -572,6 +604,41 @@ def bench_configs(args, device, stream, world, peak):
         measure(f"layer70b_{M}x{N}_k3_g8", lambda i, si=si: wl.layer70b(si, 16) if i == 0 else
                 wl.make_problem(M, N, 3, g=8, nS=wl.salient_count(0.05, N), Ks=2, batch=16, x_dtype="f16",
                                 alpha_dist="small", seed=(7, si, i)), batches=wl.BATCHES70B)
+    return out
+
+
+def bench_group_scales(args, device, stream, world, peak):
+    """The group-wise row-scale format at 4096 x 4096 (K = 2, 128 salient
+    columns with 2 bases, fp16 x): one row scale per 128 input columns
+    (fb_gemv_group_scales, G = 128), independent and dependent graphs over
+    rotating weight sets.  Algorithmic bytes as for the ordinary format with
+    the row scales K * N/G * M * 4 bytes instead of K * M * 4."""
+    import torch
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    G, nsets = 128, 48
+    ps = [wl.layer4096(seed=1 if i == 0 else (1, i)) for i in range(nsets)]
+    p0 = ps[0]
+    Ws = [fb.Weights.from_problem(p, device=device) for p in ps]
+    ars = [torch.from_numpy(np.ascontiguousarray(np.transpose(
+        wl.group_row_scales(p.K, p.M, p.N // G, seed=(43, i)), (0, 2, 1)))).to(device) for i, p in enumerate(ps)]
+    xs = [torch.from_numpy(p.x[0]).to(device) for p in ps]
+    ys = [torch.empty(p0.M, dtype=torch.float32, device=device) for _ in ps]
+    nbytes = p0.algorithmic_bytes() - 4 * p0.K * p0.M + 4 * p0.K * (p0.N // G) * p0.M
+    del ps
+    out = {"workload": "layer_4096x4096_k2_s128_G128", "G": G, "algorithmic_bytes": nbytes}
+    for name, flags in (("independent", fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT), ("dependent", fb.FB_GEMV_PDL)):
+        def body():
+            for _ in range(4):
+                for W, a, x, y in zip(Ws, ars, xs, ys):
+                    fb.fb_gemv_group_scales(W, G, x, a, y=y, flags=flags)
+        g = capture(stream, body)
+        n = max(10, args.steps // 10)
+        ms, _ = time_graph(g, stream, n, args.warmup, world)
+        del g
+        us = ms * 1e3 / (n * 4 * nsets)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"gemv_us": round(us, 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
     return out
 
 
@@ -606,13 +673,20 @@ def bench_fit(args, device, stream, peak):
             b.record(stream)
             b.synchronize()
             times.append(a.elapsed_time(b))
-    ms = statistics.median(times)
+    ms_eager = statistics.median(times)
+    # the same fit replayed from a CUDA graph (no host launch gaps)
+    graph = capture(stream, lambda: fb.fit(W, X, K, Ks, nS, sweeps))
+    gms, _ = time_graph(graph, stream, 10, 2, 1)
+    del graph
+    ms = gms / 10
     gbs = nbytes / (ms * 1e-3) / 1e9
     out = {"workload": "fit_4096x4096_k2_ks2_s128_sweeps8_t64", "ms_per_fit": round(ms, 3),
+           "ms_per_fit_eager": round(ms_eager, 3),
            "algorithmic_bytes": nbytes, "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
            "launches_per_fit": 3 + (K + Ks) * (2 * sweeps + 1) + 1,
            "note": "fb.fit: saliency, K greedy bases on R = W, gather of the salient columns, Ks bases on them; "
-                   "eager C-ABI calls, median of 5"}
+                   "ms_per_fit: the fit's launches replayed from a CUDA graph (mean of 10); eager: C-ABI calls from "
+                   "Python, median of 5"}
     if not args.no_cpu:
         import oracle.fit as ofit
         t0 = time.perf_counter()
@@ -622,47 +696,106 @@ def bench_fit(args, device, stream, peak):
     return out
 
 
-def bench_fp16_dense(args, device, stream, world, gpu_id, ours_us, ours_energy_uj):
-    """The comparison the FluxBin page draws against uncompressed weights,
-    restated per GEMV on this GPU: a dense fp16 matrix-vector product
-    (torch.mv, i.e. cuBLAS) on the same shapes, with board energy per call
-    from the power sampled during its timed region."""
+def bench_vs_fp16(args, device, stream, world, gpu_id):
+    """The comparison the FluxBin page draws against uncompressed fp16
+    weights, restated per GEMV on this GPU and like for like: on each shape,
+    our GEMV (its own workload of that shape) and a dense fp16 matrix-vector
+    product (torch.mv, i.e. cuBLAS) are each timed in the same two regimes:
+      * dependent: one call after another on one stream, each waiting for
+        the previous (ours: FB_GEMV_PDL; fp16: a plain stream of torch.mv);
+      * overlapped: independent calls allowed to run at once (ours:
+        FB_GEMV_PDL | FB_GEMV_INDEPENDENT; fp16: calls spread over 8 streams).
+    Weight copies larger than twice L2 are rotated.  Energy per call = mean
+    board power sampled during that arm's timed region x time per call."""
     import torch
-    out = {}
-    for M, N in ((4096, 4096), (11008, 4096), (8192, 8192)):
-        per = M * N * 2
-        nsets = max(2, int(2 * 126e6 // per) + 1)
-        g = torch.Generator(device=device).manual_seed(M * 7 + N)
-        Ws = [torch.randn(M, N, device=device, dtype=torch.float16, generator=g) * 0.02 for _ in range(nsets)]
-        x = torch.randn(N, device=device, dtype=torch.float16, generator=g)
-        ys = [torch.empty(M, device=device, dtype=torch.float16) for _ in range(nsets)]
-        reps = max(1, 64 // nsets)
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    l2 = 126e6
+    shapes = {
+        "4096x4096": lambda i: wl.layer4096(seed=1 if i == 0 else (1, i)),
+        "11008x4096": lambda i: wl.step7b_matrix(i, 4),
+        "8192x8192": lambda i: wl.make_problem(8192, 8192, 3, g=8, nS=wl.salient_count(0.05, 8192), Ks=2,
+                                               batch=1, x_dtype="f16", alpha_dist="small", seed=(7, 0, i)),
+    }
 
-        def body():
-            for _ in range(reps):
-                for W, y in zip(Ws, ys):
-                    torch.mv(W, x, out=y)
+    def arm(body, calls):
         graph = capture(stream, body)
-        calls = reps * nsets
-        # about half a second of timed work, for the power samples
-        one, _ = time_graph(graph, stream, 3, 1, world)
-        n = max(10, int(500.0 / max(one / 3, 1e-3)))
+        one, _ = time_graph(graph, stream, 2, 1, world)
+        n = max(10, int(400.0 / max(one / 2, 1e-3)))        # about 0.4 s of timed work for the power samples
         sampler = ClockSampler(gpu_id)
         ms, clocks = time_graph(graph, stream, n, args.warmup, world, sampler)
+        del graph
         us = ms * 1e3 / (n * calls)
-        gbs = (per + 2 * N + 2 * M) / (us * 1e-6) / 1e9
-        e = {"us": round(us, 3), "gbs": round(gbs, 1), "weight_bytes": per}
+        e = {"us": round(us, 3)}
         if clocks and clocks.get("power_w_mean"):
+            e["power_w"] = clocks["power_w_mean"]
             e["energy_uj_per_gemv"] = round(clocks["power_w_mean"] * us, 2)
-        out[f"{M}x{N}"] = e
-        del graph, Ws, ys
+        return e
+
+    out = {}
+    for name, make in shapes.items():
+        p0 = make(0)
+        M, N = p0.M, p0.N
+        per_ours = p0.algorithmic_bytes()
+        n_ours = max(2, int(2 * l2 // per_ours) + 1)
+        ps = [p0] + [make(i) for i in range(1, n_ours)]
+        Ws = [fb.Weights.from_problem(p, device=device) for p in ps]
+        xs = [torch.from_numpy(p.x[0]).to(device) for p in ps]
+        ys = [torch.empty(M, dtype=torch.float32, device=device) for _ in ps]
+        del ps
+        reps = max(1, 256 // n_ours)
+
+        def ours(flags):
+            def body():
+                for _ in range(reps):
+                    for W, x, y in zip(Ws, xs, ys):
+                        fb.fb_gemv(W, x, y=y, flags=flags)
+            return body
+        r = {"ours_bytes_per_call": per_ours}
+        r["ours_dependent"] = arm(ours(fb.FB_GEMV_PDL), reps * n_ours)
+        r["ours_overlapped"] = arm(ours(fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT), reps * n_ours)
+        del Ws, xs, ys
+
+        per_fp16 = M * N * 2
+        n_fp = max(2, int(2 * l2 // per_fp16) + 1)
+        g = torch.Generator(device=device).manual_seed(M * 7 + N)
+        Wd = [torch.randn(M, N, device=device, dtype=torch.float16, generator=g) * 0.02 for _ in range(n_fp)]
+        xd = torch.randn(N, device=device, dtype=torch.float16, generator=g)
+        yd = [torch.empty(M, device=device, dtype=torch.float16) for _ in range(n_fp)]
+        reps_fp = max(1, 128 // n_fp)
+        side = [torch.cuda.Stream(device=device) for _ in range(8)]
+
+        def fp16_dep():
+            for _ in range(reps_fp):
+                for W, y in zip(Wd, yd):
+                    torch.mv(W, xd, out=y)
+
+        def fp16_overlap():
+            cur = torch.cuda.current_stream()
+            for s in side:
+                s.wait_stream(cur)
+            k = 0
+            for _ in range(reps_fp):
+                for W, y in zip(Wd, yd):
+                    with torch.cuda.stream(side[k % len(side)]):
+                        torch.mv(W, xd, out=y)
+                    k += 1
+            for s in side:
+                cur.wait_stream(s)
+        r["fp16_bytes_per_call"] = per_fp16 + 2 * N + 2 * M
+        r["fp16_dependent"] = arm(fp16_dep, reps_fp * n_fp)
+        r["fp16_overlapped"] = arm(fp16_overlap, reps_fp * n_fp)
+        del Wd, yd
         torch.cuda.synchronize()
-    r = out["4096x4096"]
-    out["speedup_4096_ours_vs_fp16"] = round(r["us"] / ours_us, 2)
-    if ours_energy_uj and r.get("energy_uj_per_gemv"):
-        out["energy_ratio_4096_fp16_over_ours"] = round(r["energy_uj_per_gemv"] / ours_energy_uj, 2)
-    out["note"] = ("dense fp16 torch.mv (cuBLAS) on random weights of the same shapes, graph of calls over "
-                   "rotating copies larger than twice L2; energy = mean board power x time per call")
+        for regime in ("dependent", "overlapped"):
+            a, b = r[f"ours_{regime}"], r[f"fp16_{regime}"]
+            r[f"speedup_{regime}"] = round(b["us"] / a["us"], 2)
+            if "energy_uj_per_gemv" in a and "energy_uj_per_gemv" in b:
+                r[f"energy_ratio_{regime}"] = round(b["energy_uj_per_gemv"] / a["energy_uj_per_gemv"], 2)
+        out[name] = r
+    out["note"] = ("same regime on both sides: speedup = fp16 us / ours us, energy_ratio = fp16 energy / ours; "
+                   "ours = the build's workload of that shape (4096: K=2 g=4 128 salient; 11008x4096: 7B gate, "
+                   "K=2 3% salient; 8192: K=3 g=8 5% salient); fp16 = torch.mv on random weights")
     return out
 
 
