@@ -172,11 +172,12 @@ FB_API size_t fb_gemv_workspace_bytes(const fb_weights *W, int batch);
                           kernel still completes only after the previous one,
                           so ordering with later work is unchanged. */
 
-#define FB_GEMV_TEST_WAIT_TIMEOUT 0x80000000u /* for tests of the failure path:
-                          the kernel issues no weight copy, so its bounded wait
-                          for one runs out (about 0.2 s); it then writes NaN
-                          into every row and raises bit 0 of fb_device_errors.
-                          The context stays usable. */
+#define FB_GEMV_TEST_WAIT_TIMEOUT 0x80000000u /* for tests of the failure path
+                          (batch-1 calls): no CTA sends its row partials, so
+                          every CTA's bounded wait for them runs out (about
+                          0.2 s); it then writes NaN into the rows it owns and
+                          raises bit 0 of fb_device_errors.  The context stays
+                          usable. */
 
 /* fb_gemv: y[i] = sum_j W_hat[i][j] * x[j] for i < M (batch 1), fp32 out,
  * overwriting y (beta = 0).  x: N elements of type t (2- or 4-byte aligned);
@@ -185,14 +186,19 @@ FB_API size_t fb_gemv_workspace_bytes(const fb_weights *W, int batch);
  * optionally | FB_GEMV_TEST_WAIT_TIMEOUT; anything else is
  * FB_ERR_INVALID_VALUE.  Table entries and all sums are
  * fp32.  Deterministic: the same inputs give the same bits on every run.
- * Weight copies are waited for with a bound (about 0.2 s); a kernel that
+ * The CTAs of a thread-block cluster exchange row partials through shared
+ * memory; each waits for its share with a bound (about 0.2 s), and one that
  * gives up writes NaN into the rows it owns and raises bit 0 of
  * fb_device_errors. */
 FB_API fb_status fb_gemv(const fb_weights *W, const void *x, fb_dtype t, float *y, void *ws,
                   size_t ws_bytes, unsigned flags, void *stream);
 
 /* fb_gemv_batched: Y[b*ldy + i] = sum_j W_hat[i][j] * X[b*ldx + j] for
- * b < batch (1 <= batch <= 64), i < M.  ldx >= N, ldy >= M. */
+ * b < batch (1 <= batch <= 64), i < M.  ldx >= N, ldy >= M.  The tokens are
+ * processed in passes of up to 8: within a pass, each weight word is read
+ * from memory once and applied to every token's tables.  Per token the
+ * result has the same properties as fb_gemv's (fp32 sums, deterministic,
+ * same tolerance). */
 FB_API fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtype t, int batch, int ldx,
                           float *Y, int ldy, void *ws, size_t ws_bytes, unsigned flags,
                           void *stream);
@@ -236,15 +242,16 @@ FB_API fb_status fb_gemv_group_scales(const fb_weights *W, int G, const void *x,
  * memory bytes per CTA, out[5] = virtual panels (256-column panels x bases).
  * out must hold 6 ints.  Returns FB_OK, or FB_ERR_INVALID_VALUE for invalid
  * weights, batch, sms or flags.  Tuning aid: the environment variable
- * FB_PLAN="C,cpb", read when a plan is first made for a shape, forces the
+ * FB_PLAN="C,cpb[,n]", read when a plan is first made for a shape, forces the
  * cluster size and row block (clamped to what the matrix and shared memory
- * allow). */
+ * allow); the optional n is, for batch-1 calls, 16 to use 16-warp CTAs (one
+ * per SM) and, for batched calls, the tokens per pass (even, at most 16). */
 FB_API fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned flags, int sms, int *out);
 
 /* fb_device_errors: synchronises the current device, then stores in *flags
- * the error bits GEMV kernels have raised since the last clear (bit 0: a
- * kernel gave up a bounded wait for one of its weight copies; the rows of
- * that CTA were written as NaN), and clears them when clear != 0.  Returns
+ * the error bits GEMV kernels have raised since the last clear (bit 0: a CTA
+ * gave up its bounded wait for the row partials of its cluster; the rows it
+ * owns were written as NaN), and clears them when clear != 0.  Returns
  * FB_ERR_INVALID_VALUE for a null flags, FB_ERR_CUDA if the device reports an
  * error, else FB_OK. */
 FB_API fb_status fb_device_errors(unsigned int *flags, int clear);

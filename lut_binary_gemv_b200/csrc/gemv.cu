@@ -8,29 +8,34 @@
 // global or salient; the matrix has V of them.  Rows come in chunks of 32,
 // one row per lane; an "item" is one chunk of one virtual panel (32 rows x
 // <= 32 bytes).  A thread-block cluster of C CTAs owns one block of cpb
-// chunks; CTA j of the cluster takes a contiguous, balanced slice of the V
-// virtual panels, so the cluster covers every column of its rows.
+// chunks; CTA j of the cluster takes a contiguous slice of the V virtual
+// panels (balanced by their lookup work), so the cluster covers every column
+// of its rows.
 //
-// Per CTA (16 warps, or 8 for dependent calls; warp w owns chunks w and
-// w + warps of the row block):
-//   1. before the programmatic-launch wait: the weights of the first panels
-//      start streaming into shared-memory slots (one bulk asynchronous copy
-//      per panel of the row block, completion on an mbarrier), and the row
-//      scales and per-panel descriptors are staged in shared memory;
-//   2. per panel, all 256 threads build its byte tables in shared memory
+// stream_kernel (batch 1; 8 warps, two CTAs per SM, or 16 warps, one):
+//   1. the words of the CTA's first two panels are loaded straight into
+//      registers (each lane its rows' bytes, 128-bit loads), with the row
+//      scales; for calls that depend on the previous kernel this, and an L2
+//      prefetch of the rest of the slice, happens before the
+//      programmatic-launch wait, and x is read after it;
+//   2. per panel, the CTA builds the panel's byte tables in shared memory
 //      (LUT-BSF: z = alpha_c * x, salient panels reading x[s_idx[t]] -- the
 //      virtual columnar mapping -- and for each group of 8 columns the 256
 //      sums sum_t (bit t of b ? +z_t : -z_t), each the sum of the two 4-column
 //      tables of its nibbles), double-buffered, one CTA barrier per panel;
-//   3. each lane walks its row's 32 bytes: one `prmt` merges a weight byte and
+//      meanwhile the words of the panel after next load into the register
+//      set the previous panel used;
+//   3. each lane walks its row's bytes: one `prmt` merges a weight byte and
 //      the lane's column offset into a table address, one shared load fetches
 //      the partial sum, packed fp32x2 adds accumulate (a gather-add, no tensor
 //      cores); each item's sum is scaled by alpha_r once (alpha_r applied in
 //      the reduction) and added to the row's partial;
-//   4. each CTA pushes its row partials into the shared memory of the CTA
-//      that owns those rows, the cluster synchronises once, and each owner
-//      sums its C inbox slots in rank order and writes y.  No workspace, no
-//      atomics; deterministic.
+//   4. each row partial is sent to the cluster CTA that owns the row as an
+//      asynchronous remote store completing on the owner's barrier; the
+//      owner waits (bounded) for all of them and sums its C slots in rank
+//      order.  No workspace, no atomics; deterministic.
+// batched_kernel (several tokens): the same, with each panel's words applied
+// to every token of a pass in turn (one weight pass per pass of tokens).
 //
 // Byte tables: entry b of byte group q (columns 8q .. 8q+7 of the panel) is
 // at b*256 + 4q bytes; the two buffers interleave, the second at +128.  Lane
@@ -59,21 +64,8 @@ namespace fb {
 namespace {
 
 constexpr int kMaxCluster = 16;   // 16: non-portable cluster size (B200 allows it)
-constexpr int kMaxSlotCluster = 8;   // gemv_kernel's plans stay within the portable size
 constexpr int kMaxGroup = 4;            // matrices in one grouped call
-// Two CTA shapes.  16 warps, one CTA per SM, up to 32 chunks per row block
-// and three weight slots: calls flagged independent (fewest table builds per
-// row).  8 warps, two CTAs per SM, up to 16 chunks and two slots: dependent
-// calls (twice the CTAs in one wave, shorter panel lists per CTA).  Both give
-// each warp two chunks of every panel.
-template <int NW>
-struct Shape {
-    static constexpr int kSlots = NW == 16 ? 3 : 2;
-    static constexpr int kMinBlocks = 16 / NW;     // CTAs per SM the registers allow
-};
 constexpr size_t kMaxDynSmem = 225 * 1024;   // dynamic shared memory per CTA
-constexpr size_t kSmemPerSM = 228 * 1024;
-constexpr size_t kStaticSmem = 1024;          // the kernel's static shared memory, rounded up
 constexpr unsigned kKnownFlags = FB_GEMV_PDL | FB_GEMV_INDEPENDENT | FB_GEMV_TEST_WAIT_TIMEOUT;
 
 struct GemvArgs {
@@ -129,17 +121,6 @@ __device__ __forceinline__ void mbar_init(uint32_t bar) {
 }
 __device__ __forceinline__ void mbar_init_fence() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-// One copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
-// global memory into this CTA's shared memory; the barrier's phase completes
-// when the bytes have landed.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .b64 st;\n\t"
-        "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%2], %1;\n\t"
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%3], %1, [%2];\n\t}"
-        ::"r"(dst), "r"(bytes), "r"(bar), "l"(src)
-        : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -353,35 +334,50 @@ __device__ __forceinline__ PanelDesc panel_desc(const GemvArgs &a, int v) {
     return d;
 }
 
-// Column c of a panel: its scale alpha_c and the column of x it reads (-1:
-// none: the other half of a half-panel, and the columns past a narrow
-// panel's width, which build all-zero table columns).  With kDup, the
-// columns past a narrow panel's width (Bp < 32 byte groups) instead repeat
-// its columns, floor(32 / Bp) copies in all, so lanes of a warp that share a
-// byte group can read different copies (narrow_offsets_dup).
-template <bool kDup = false>
-__device__ __forceinline__ void column_source(const GemvArgs &a, const PanelDesc &d, int c, float &ac, int &xi) {
-    ac = 0.0f;
-    xi = -1;
+// Column staging in two phases, so no thread waits on the salient column
+// index while it stages: stage_column issues the loads of column c's scale
+// and -- for a global column -- of its x; for a salient column it loads the
+// index s_idx (xi = kPendingIndex, the raw index in x), and resolve_column,
+// one panel later, turns the index into the x column and issues that load.
+constexpr int kPendingIndex = -2;
+
+struct Staged {
+    float ac;     // alpha_c of the column (0: none)
+    uint32_t x;   // stored bits of x[xi]; or the raw salient index while xi == kPendingIndex
+    int xi;       // column of x, -1 (none) or kPendingIndex
+};
+
+template <int XT, bool kDup>
+__device__ __forceinline__ void stage_column(const GemvArgs &a, const PanelDesc &d, int c, size_t xoff, bool read_x,
+                                             Staged &t) {
+    t.ac = 0.0f;
+    t.xi = -1;
+    t.x = 0;
     const int w = desc_bp(d) * 8;
     if (c >= w) {
         if (!kDup || c >= (kPanelCols / w) * w) return;
         c -= (c / w) * w;
     }
     const int half = desc_half(d);
-    if (half && (c >> 7) != half - 1) return;   // a half-panel: the other half's columns build zeros
+    if (half && (c >> 7) != half - 1) return;
     const int col = d.col0 + c;
     if (!desc_sal(d)) {
-        xi = col;
-        if (d.ac)
-            ac = __ldg(d.ac + col);
-        else
-            ac = 1.0f;
+        t.xi = col;
+        t.ac = d.ac ? __ldg(d.ac + col) : 1.0f;
+        if (read_x) t.x = load_x_bits<XT>(a.x, xoff + col);
     } else if (col < a.nS) {
-        ac = __ldg(d.ac + col);
-        const uint32_t jx = __ldg(a.s_idx + col);
-        xi = jx < (uint32_t)a.N ? (int)jx : -1;   // an invalid index contributes 0
+        t.ac = __ldg(d.ac + col);
+        t.x = __ldg(a.s_idx + col);
+        t.xi = kPendingIndex;
     }
+}
+
+template <int XT>
+__device__ __forceinline__ void resolve_column(const GemvArgs &a, size_t xoff, Staged &t) {
+    if (t.xi != kPendingIndex) return;
+    const uint32_t jx = t.x;
+    t.xi = jx < (uint32_t)a.N ? (int)jx : -1;   // an invalid index contributes 0
+    t.x = t.xi >= 0 ? load_x_bits<XT>(a.x, xoff + t.xi) : 0u;
 }
 
 // Column offsets of a full panel: byte j of offp[m] = 4 * ((lane + 4m + j) mod 32).
@@ -400,25 +396,6 @@ __device__ __forceinline__ void full_offsets(int lane, uint32_t (&offp)[8]) {
 struct Offsets {
     uint32_t w[8];
 };
-__device__ __noinline__ Offsets narrow_offsets(int lane, int Bp) {
-    Offsets o;
-    const int r = lane % Bp;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int u = 4 * m + jj;
-            int q = r + u;
-            q = q >= Bp ? q - Bp : q;
-            q = u < Bp ? q : 31;
-            word |= (uint32_t)(4 * q) << (8 * jj);
-        }
-        o.w[m] = word;
-    }
-    return o;
-}
-
 // Column offsets of a narrow panel (Bp < 32) whose table repeats its byte
 // groups (column_source<true>): lane l reads copy (l / Bp) mod floor(32/Bp),
 // so byte j of word m = 4 * ((l mod Bp + u) mod Bp + Bp * copy) for position
@@ -531,294 +508,22 @@ __device__ __forceinline__ void build_byte_table(const float *zp, float *T, int 
         for (int v = 0; v < 16; ++v) col[(16 * s2 + v) * 64] = __fadd_rn(lo[v], hi[s2]);
 }
 
-// Set (bit 0) when a kernel gave up waiting for a weight copy; the rows of
-// that CTA are then written as NaN.  Read and cleared by fb_device_errors.
+// Set (bit 0) when a CTA gave up waiting for its cluster's row partials;
+// the rows it owns are then written as NaN.  Read and cleared by
+// fb_device_errors.
 __device__ unsigned int g_error_flags;
 
-// The row's words of one item of a narrow panel (Bp < 32) from its slot
-// (the block's bytes in the packed layout); positions past Bp are zero.
+// One lane's words of one item: position u in byte u % 4 of w[u / 4].
 struct Words {
     uint32_t w[8];
 };
-__device__ __noinline__ Words read_item_narrow(const uint8_t *slot, int Bp, int lane) {
-    Words r;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) r.w[m] = 0;
-    if (Bp == 16) {
-        const uint4 x0 = *reinterpret_cast<const uint4 *>(slot + 16 * lane);
-        r.w[0] = x0.x; r.w[1] = x0.y; r.w[2] = x0.z; r.w[3] = x0.w;
-    } else {
-#pragma unroll
-        for (int m = 0; m < 7; ++m)
-            if (m < Bp / 4) r.w[m] = *reinterpret_cast<const uint32_t *>(slot + 128 * m + 4 * lane);
-    }
-    return r;
-}
-
-// The row's words of one item of a full panel from its slot.
-__device__ __forceinline__ void read_item_full(const uint8_t *slot, int lane, uint32_t (&w)[8]) {
-    const uint4 x0 = *reinterpret_cast<const uint4 *>(slot + 16 * lane);
-    const uint4 x1 = *reinterpret_cast<const uint4 *>(slot + 512 + 16 * lane);
-    w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
-    w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
-}
-
-// Shared-memory layout of one CTA (bytes): two interleaved byte tables |
-// z of two panels | kSlots weight slots of cpb KiB | row scales [KB][R] |
-// row partials [R] | cluster inbox [R + C].
+// Shared memory of the byte tables (two interleaved buffers) and of the z
+// values of two panels.
 constexpr int kTableBytes = 65536;
 constexpr int kZBytes = 2 * kPanelCols * 4;
-constexpr int kItemsPerWarp = 2;
-
-template <int XT, int NW>
-__global__ void __launch_bounds__(NW * 32, Shape<NW>::kMinBlocks) gemv_kernel(const __grid_constant__ GemvArgs args) {
-    constexpr int kNW = NW, kSlots = Shape<NW>::kSlots;
-    extern __shared__ __align__(128) float smem_f[];
-    __shared__ __align__(8) unsigned long long s_bar[kSlots];
-    // The launch's parameter block is new to every SM's constant cache, and the
-    // kernel would touch its fields one after another, each a miss; one
-    // parallel copy into shared memory pays that latency once.
-    __shared__ __align__(16) GemvArgs s_args;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // (the per-matrix table of grouped calls stays in the parameter block)
-    static_assert(offsetof(GemvArgs, mats) % 4 == 0, "parameter block copied as words");
-    for (int i = tid; i < (int)(offsetof(GemvArgs, mats) / 4); i += blockDim.x)
-        reinterpret_cast<int *>(&s_args)[i] = reinterpret_cast<const int *>(&args)[i];
-    if (tid == 0) {
-#pragma unroll
-        for (int s2 = 0; s2 < kSlots; ++s2) mbar_init(smem_addr(&s_bar[s2]));
-        mbar_init_fence();
-    }
-    if (args.group > 1) {   // a grouped call: this CTA's matrix
-        __syncthreads();
-        if (tid == 0) {
-            int m = 0;
-            while (m + 1 < s_args.group && (int)blockIdx.y >= s_args.rb_start[m + 1]) ++m;
-            const GemvArgs::Mat &mt = args.mats[m];
-            s_args.planes = mt.planes;
-            s_args.alpha_r = mt.alpha_r;
-            s_args.alpha_c = mt.alpha_c;
-            s_args.s_planes = mt.s_planes;
-            s_args.s_alpha_r = mt.s_alpha_r;
-            s_args.s_alpha_c = mt.s_alpha_c;
-            s_args.s_idx = mt.s_idx;
-            s_args.y = mt.y;
-            s_args.M = mt.M;
-            s_args.M_pad = mt.M_pad;
-            s_args.nchunks = mt.nchunks;
-            s_args.rb_base = s_args.rb_start[m];
-        }
-    }
-    __syncthreads();
-    const GemvArgs &a = s_args;
-    cg::cluster_group cluster = cg::this_cluster();
-    const int j = (int)cluster.block_rank();
-    const int rb = (int)blockIdx.y - a.rb_base, b = blockIdx.z;
-    const int vb = a.vsplit[j], n_v = a.vsplit[j + 1] - a.vsplit[j];
-    const int cpb = a.cpb, R = cpb * kChunkRows;
-    const int c_first = rb * cpb;
-    const int nvalid = min(cpb, a.nchunks - c_first);   // chunks of this row block inside the matrix
-    const int KB = a.K + a.Ks;                          // bases with row scales: global, then salient
-    const bool independent = (a.flags & FB_GEMV_INDEPENDENT) != 0;
-    const size_t xoff = (size_t)b * a.ldx;
-    const int slot_bytes = cpb * 1024;
-
-    float *tables = smem_f;
-    float *zbuf = smem_f + kTableBytes / 4;
-    uint8_t *slots = reinterpret_cast<uint8_t *>(smem_f) + kTableBytes + kZBytes;
-    float *s_ar = reinterpret_cast<float *>(slots + kSlots * slot_bytes);
-    float *pw = s_ar + KB * R;
-    float *part = pw + R;
-    PanelDesc *s_desc = reinterpret_cast<PanelDesc *>(part + ((R + kMaxCluster + 1) & ~1));
-    const uint32_t slots_s = smem_addr(slots), bar_s = smem_addr(&s_bar[0]);
-
-    // ---- 1. weight copies and row scales, before the wait -------------------
-    // Panel vi's blocks of this row block are contiguous: one bulk copy into
-    // slot vi % kSlots, issued by thread 0 kSlots - 1 panels ahead of use.
-    uint32_t pending = 0, pend_par = 0;   // thread 0: slots with a copy in flight, its phase parity
-    auto issue = [&](int vi, const PanelDesc &d) {
-        if (a.flags & FB_GEMV_TEST_WAIT_TIMEOUT) return;   // tests: no copy, so every wait for one runs out
-        const int s2 = vi % kSlots;
-        const uint32_t blk = 32u * (uint32_t)desc_bp(d);
-        bulk_load(slots_s + s2 * slot_bytes, d.pl + (size_t)blk * c_first, blk * (uint32_t)nvalid, bar_s + 8 * s2);
-        pending |= 1u << s2;
-        pend_par = (pend_par & ~(1u << s2)) | ((uint32_t)(vi / kSlots) & 1u) << s2;
-    };
-    if (tid == 0)
-        for (int v = 0; v < kSlots - 1 && v < n_v; ++v) issue(v, panel_desc(a, vb + v));
-    for (int t = tid; t < n_v; t += blockDim.x) s_desc[t] = panel_desc(a, vb + t);
-
-    // column data of one panel: thread t stages column t
-    // Two register sets, for panels of even and odd index: panel p is staged
-    // two panels before its z is written (the loop below is unrolled by two,
-    // so the set is chosen at compile time).
-    struct Staged {
-        float ac;
-        uint32_t x;
-        int xi;
-    };
-    Staged st[2] = {{0.0f, 0u, -1}, {0.0f, 0u, -1}};
-    auto stage = [&](Staged &t, const PanelDesc &d, bool read_x) {
-        t.x = 0;
-        if (tid >= kPanelCols) return;
-        column_source(a, d, tid, t.ac, t.xi);
-        if (read_x && t.xi >= 0) t.x = load_x_bits<XT>(a.x, xoff + t.xi);
-    };
-    auto z_of = [&](const Staged &t) { return t.xi >= 0 ? __fmul_rn(t.ac, x_value<XT>(t.x)) : 0.0f; };
-    if (n_v > 0) stage(st[0], panel_desc(a, vb), independent);
-    griddep_launch_dependents();
-    // the row block's row scales, every base (rows past M: 0); a thread's
-    // loads are issued in batches of kArBatch before any is stored, so they
-    // cost one memory latency per batch rather than one each
-    constexpr int kArBatch = 8;
-    for (int t0 = 0; t0 < KB * R; t0 += kArBatch * (int)blockDim.x) {
-        float v[kArBatch];
-#pragma unroll
-        for (int u = 0; u < kArBatch; ++u) {
-            const int t = t0 + u * (int)blockDim.x + tid;
-            const int kb = t / R, r = t - kb * R, row = c_first * kChunkRows + r;
-            const float *src = row_scales(a, kb);
-            v[u] = t < KB * R && row < a.M ? __ldg(src + row) : 0.0f;
-        }
-#pragma unroll
-        for (int u = 0; u < kArBatch; ++u) {
-            const int t = t0 + u * (int)blockDim.x + tid;
-            if (t < KB * R) s_ar[t] = v[u];
-        }
-    }
-
-    // ---- 2. activations (may be the previous kernel's output) --------------
-    if (!independent) {
-        griddep_wait();
-        if (st[0].xi >= 0) st[0].x = load_x_bits<XT>(a.x, xoff + st[0].xi);
-    }
-    if (tid < kPanelCols) zbuf[tid] = z_of(st[0]);
-    __syncthreads();   // z of panel 0, panel descriptors and row scales written
-    if (n_v > 1) stage(st[1], s_desc[1], true);
-    if (n_v > 2) stage(st[0], s_desc[2], true);
-
-    // column offsets of a full panel (narrow panels compute theirs)
-    uint32_t off_full[8];
-    full_offsets(lane, off_full);
-
-    // ---- 3. per panel: its byte tables, then this warp's chunks -------------
-    // Warp w owns chunks w + kNW * i of the row block; each lane keeps its
-    // rows' partial sums and current row scales in registers.  The barrier of
-    // panel vi also ends every warp's reads of panel vi - 1, whose slot then
-    // takes panel vi + kSlots - 1.
-    bool failed = false;
-    float racc[kItemsPerWarp], rar[kItemsPerWarp];
-#pragma unroll
-    for (int it = 0; it < kItemsPerWarp; ++it) racc[it] = rar[it] = 0.0f;
-    int kb_cur = -1, sl = 0;   // sl = vi % kSlots
-    // One panel; the table buffer is a compile-time constant in each of the
-    // two copies, so table addresses fold into the shared loads.
-    auto panel = [&](auto bufc, int vi) {
-        constexpr int buf = decltype(bufc)::value;
-        const int Bp = desc_bp(s_desc[vi]), kb = s_desc[vi].kb;
-        bool ok = !failed;
-        if (ok) {
-            const uint32_t par = (uint32_t)(vi / kSlots) & 1u;
-            ok = mbar_try_wait(bar_s + 8 * sl, par) || mbar_wait_bounded(bar_s + 8 * sl, par);
-        }
-        if (tid == 0 && ok) pending &= ~(1u << sl);
-        float *tb = tables + 32 * buf;
-        build_byte_table<NW>(zbuf + buf * kPanelCols, tb, warp, lane);
-        if (vi + 1 < n_v && tid < kPanelCols)   // z of the next panel into the other buffer
-            zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
-        if (vi + 3 < n_v) stage(st[buf ^ 1], s_desc[vi + 3], true);
-        // tables of panel vi complete; every warp done with panel vi - 1
-        failed = __syncthreads_or(!ok) != 0;
-        if (failed) return;
-        if (tid == 0 && vi + kSlots - 1 < n_v) issue(vi + kSlots - 1, s_desc[vi + kSlots - 1]);
-        if (kb != kb_cur) {   // a new base: its row scales
-            kb_cur = kb;
-#pragma unroll
-            for (int it = 0; it < kItemsPerWarp; ++it) {
-                const int cl = warp + kNW * it;
-                if (cl < cpb) rar[it] = s_ar[kb_cur * R + cl * kChunkRows + lane];
-            }
-        }
-        const uint8_t *slot = slots + sl * slot_bytes;
-        sl = sl + 1 == kSlots ? 0 : sl + 1;
-        static_assert(kItemsPerWarp == 2, "the full-panel path looks up a warp's two items together");
-        if (Bp == 32 && warp + kNW < nvalid) {   // both items: interleaved
-            uint32_t w0[8], w1[8];
-            read_item_full(slot + warp * 1024, lane, w0);
-            read_item_full(slot + (warp + kNW) * 1024, lane, w1);
-            float s0, s1;
-            lookup_rows2(w0, w1, off_full, tb, s0, s1);
-            racc[0] = __fadd_rn(racc[0], __fmul_rn(rar[0], s0));
-            racc[1] = __fadd_rn(racc[1], __fmul_rn(rar[1], s1));
-        } else if (Bp == 32) {
-            if (warp < nvalid) {
-                uint32_t w[8];
-                read_item_full(slot + warp * 1024, lane, w);
-                racc[0] = __fadd_rn(racc[0], __fmul_rn(rar[0], lookup_row(w, off_full, tb)));
-            }
-        } else {
-            const Offsets o = narrow_offsets(lane, Bp);
-#pragma unroll 1
-            for (int it = 0; it < kItemsPerWarp; ++it) {
-                const int cl = warp + kNW * it;
-                if (cl < nvalid) {
-                    const Words r = read_item_narrow(slot + cl * 32 * Bp, Bp, lane);
-                    const float sum = lookup_row(r.w, o.w, tb);
-#pragma unroll
-                    for (int i2 = 0; i2 < kItemsPerWarp; ++i2)
-                        if (i2 == it) racc[i2] = __fadd_rn(racc[i2], __fmul_rn(rar[i2], sum));
-                }
-            }
-        }
-    };
-#pragma unroll 1
-    for (int vi = 0; vi < n_v; vi += 2) {
-        panel(std::integral_constant<int, 0>{}, vi);
-        if (vi + 1 < n_v) panel(std::integral_constant<int, 1>{}, vi + 1);
-    }
-#pragma unroll
-    for (int it = 0; it < kItemsPerWarp; ++it) {
-        const int cl = warp + kNW * it;
-        if (cl < cpb) pw[cl * kChunkRows + lane] = racc[it];
-    }
-    if (failed && tid == 0) {
-        // Wait (bounded) for the copies still in flight, so none lands after
-        // the CTA has gone, then flag the failure.
-        for (int s2 = 0; s2 < kSlots; ++s2)
-            if (pending & (1u << s2)) mbar_wait_bounded(bar_s + 8 * s2, (pend_par >> s2) & 1u);
-        atomicOr(&g_error_flags, 1u);
-    }
-
-    // ---- 4. the cluster's row partials, in a fixed order --------------------
-    // Rows are owned in runs of Rq: rank o sums rows [o*Rq, min((o+1)*Rq, R)).
-    // Every CTA pushes its row partials into the owner's inbox (slot = its
-    // own rank), one cluster barrier makes them visible, and each owner adds
-    // its inbox in rank order.  After the barrier no CTA touches another's
-    // shared memory, so none has to wait for the others before exiting.
-    const int Rq = (R + a.C - 1) / a.C;
-    __syncthreads();
-    for (int r = tid; r < R; r += blockDim.x) {
-        const float sum = failed ? __int_as_float(0x7fc00000) : pw[r];
-        const int owner = r / Rq;
-        float *inbox = cluster.map_shared_rank(part, owner);
-        inbox[j * Rq + (r - owner * Rq)] = sum;
-    }
-    cluster.sync();
-    for (int i = tid; i < Rq; i += blockDim.x) {
-        const int r = j * Rq + i;
-        if (r >= R) break;
-        float sum = part[i];
-        for (int jj = 1; jj < a.C; ++jj) sum = __fadd_rn(sum, part[jj * Rq + i]);
-        const int row = c_first * kChunkRows + r;
-        if (row < a.M) a.y[(size_t)b * a.ldy + row] = sum;
-    }
-    if (independent) griddep_wait();   // complete only after the previous kernel
-}
-
 // ---- The streaming kernel: weights straight into registers --------------
 //
-// Same work units, tables, lookups and cluster reduction as gemv_kernel, but
-// the packed weights are not staged in shared memory: each lane loads its
+// The packed weights are not staged in shared memory: each lane loads its
 // rows' words of the panel after next with 128-bit loads into one of two
 // register sets while it looks up the current panel from the other, so a
 // weight byte costs shared-memory bandwidth only for its table lookup.  8
@@ -865,9 +570,10 @@ __device__ __noinline__ Words load_item_narrow(const uint8_t *blk, int Bp, int l
 constexpr int kStreamWarps = 8;
 constexpr int kDescRing = 8;   // panel descriptors kept in shared memory (a ring)
 
-template <int XT, int I>
-__global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_kernel(const __grid_constant__ GemvArgs args) {
-    constexpr int NW = kStreamWarps;
+template <int XT, int NW, int I>
+__global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_constant__ GemvArgs args) {
+    static_assert(NW == 8 || NW == 16, "8 warps (two CTAs per SM) or 16 (one)");
+    constexpr bool kAllStage = NW * 32 == kPanelCols;   // every thread stages a column
     extern __shared__ __align__(128) float smem_f[];
     __shared__ __align__(16) GemvArgs s_args;
     __shared__ __align__(16) PanelDesc s_ring[kDescRing];
@@ -928,60 +634,51 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_kernel(const __gr
     }
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-    // ---- 1. before the wait: the first two panels' words, their row
-    // scales, the column sources of panel 0 (and its x when independent) --
-    uint32_t wA[I][8], wB[I][8];
-    float rarA[I], rarB[I];
-    auto load_panel = [&](uint32_t (&w)[I][8], float (&rar)[I], const PanelDesc &d) {
+    // ---- 1. before the wait: panel 0's words and row scales, the column
+    // sources of panel 0 (and its x when independent) ----------------------
+    // One register set: right after an item's lookups, its registers take
+    // the same item of the next panel, so each load has a panel's time to
+    // land (two alternating sets would give no more lead).
+    uint32_t w[I][8];
+    float rar[I];
+    auto load_item = [&](int i, const PanelDesc &d) {
         const int Bp = desc_bp(d);
         const size_t blk = 32u * (unsigned)Bp;
-        const float *src = row_scales(a, d.kb);
+        const int cl = warp + NW * i;
+        const int row = (c_first + cl) * kChunkRows + lane;
+        rar[i] = cl < nvalid && row < a.M ? __ldg(row_scales(a, d.kb) + row) : 0.0f;
+        if (cl < nvalid) {
+            const uint8_t *p = d.pl + blk * (size_t)(c_first + cl);
+            if (Bp == 32) {
+                const uint4 x0 = ldg_stream(p + 16 * lane), x1 = ldg_stream(p + 512 + 16 * lane);
+                w[i][0] = x0.x; w[i][1] = x0.y; w[i][2] = x0.z; w[i][3] = x0.w;
+                w[i][4] = x1.x; w[i][5] = x1.y; w[i][6] = x1.z; w[i][7] = x1.w;
+            } else {
+                const Words r = load_item_narrow(p, Bp, lane);
 #pragma unroll
-        for (int i = 0; i < I; ++i) {
-            const int cl = warp + NW * i;
-            const int row = (c_first + cl) * kChunkRows + lane;
-            rar[i] = cl < nvalid && row < a.M ? __ldg(src + row) : 0.0f;
-            if (cl < nvalid) {
-                const uint8_t *p = d.pl + blk * (size_t)(c_first + cl);
-                if (Bp == 32) {
-                    const uint4 x0 = ldg_stream(p + 16 * lane), x1 = ldg_stream(p + 512 + 16 * lane);
-                    w[i][0] = x0.x; w[i][1] = x0.y; w[i][2] = x0.z; w[i][3] = x0.w;
-                    w[i][4] = x1.x; w[i][5] = x1.y; w[i][6] = x1.z; w[i][7] = x1.w;
-                } else {
-                    const Words r = load_item_narrow(p, Bp, lane);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) w[i][m] = r.w[m];
-                }
+                for (int m = 0; m < 8; ++m) w[i][m] = r.w[m];
             }
         }
     };
     if (tid < kDescRing - 4 && tid < n_v) s_ring[tid] = panel_desc(a, vb + tid);
-    struct Staged {
-        float ac;
-        uint32_t x;
-        int xi;
-    };
     Staged st[2] = {{0.0f, 0u, -1}, {0.0f, 0u, -1}};
     auto stage = [&](Staged &t, const PanelDesc &d, bool read_x) {
-        t.x = 0;
-        column_source<true>(a, d, tid, t.ac, t.xi);
-        if (read_x && t.xi >= 0) t.x = load_x_bits<XT>(a.x, xoff + t.xi);
+        if (kAllStage || tid < kPanelCols) stage_column<XT, true>(a, d, tid, xoff, read_x, t);
     };
+    auto resolve = [&](Staged &t) { resolve_column<XT>(a, xoff, t); };
     auto z_of = [&](const Staged &t) { return t.xi >= 0 ? __fmul_rn(t.ac, x_value<XT>(t.x)) : 0.0f; };
     PanelDesc d1;
     if (n_v > 0) {
         const PanelDesc d0 = panel_desc(a, vb);
-        load_panel(wA, rarA, d0);
+#pragma unroll
+        for (int i = 0; i < I; ++i) load_item(i, d0);
         stage(st[0], d0, independent);
     }
-    if (n_v > 1) {
-        d1 = panel_desc(a, vb + 1);
-        load_panel(wB, rarB, d1);
-    }
+    if (n_v > 1) d1 = panel_desc(a, vb + 1);
     if (!independent) {
         // the rest of the slice into L2 while the previous kernel finishes
         if (tid == 0) {
-            for (int v = 2; v < min(n_v, 8); ++v) {
+            for (int v = 1; v < min(n_v, 8); ++v) {
                 const PanelDesc d = panel_desc(a, vb + v);
                 const uint32_t blk = 32u * (uint32_t)desc_bp(d);
                 prefetch_l2(d.pl + (size_t)blk * c_first, blk * (uint32_t)nvalid);
@@ -991,7 +688,9 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_kernel(const __gr
         if (st[0].xi >= 0) st[0].x = load_x_bits<XT>(a.x, xoff + st[0].xi);
     }
     if (n_v > 1) stage(st[1], d1, true);   // x of panel 1 in flight with panel 0's
-    zbuf[tid] = z_of(st[0]);
+    resolve(st[0]);
+    if (n_v > 1) resolve(st[1]);
+    if (kAllStage || tid < kPanelCols) zbuf[tid] = z_of(st[0]);
     __syncthreads();   // z of panel 0 and the first descriptors written
     if (n_v > 2) stage(st[0], s_ring[2], true);
 
@@ -1003,15 +702,18 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_kernel(const __gr
     for (int i = 0; i < I; ++i) racc[i] = 0.0f;
 
     // ---- 2. per panel: tables, then this warp's items ----------------------
-    auto panel = [&](auto bufc, int vi, uint32_t (&w)[I][8], float (&rar)[I]) {
+    auto panel = [&](auto bufc, int vi) {
         constexpr int buf = decltype(bufc)::value;
         const int Bp = desc_bp(s_ring[vi % kDescRing]);
         float *tb = tables + 32 * buf;
         build_byte_table<NW>(zbuf + buf * kPanelCols, tb, warp, lane);
-        if (vi + 1 < n_v) zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
+        if (vi + 1 < n_v && (kAllStage || tid < kPanelCols)) zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
         if (vi + 3 < n_v) stage(st[buf ^ 1], s_ring[(vi + 3) % kDescRing], true);
+        if (vi + 2 < n_v) resolve(st[buf]);   // panel vi + 2, staged one panel ago
         if (tid == 0 && vi + 4 < n_v) s_ring[(vi + 4) % kDescRing] = panel_desc(a, vb + vi + 4);
         __syncthreads();   // tables of panel vi complete; every warp done with panel vi - 1
+        const bool more = vi + 1 < n_v;
+        const PanelDesc &nd = s_ring[(vi + 1) % kDescRing];   // the next panel (its items load here)
         if (Bp == 32) {
 #pragma unroll
             for (int i = 0; i < I; i += 2) {
@@ -1024,20 +726,25 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_kernel(const __gr
                 } else if (c0 < nvalid) {
                     racc[i] = __fadd_rn(racc[i], __fmul_rn(rar[i], lookup_row(w[i], off_full, tb)));
                 }
+                if (more) {
+                    load_item(i, nd);
+                    if (i + 1 < I) load_item(i + 1, nd);
+                }
             }
         } else {
             const Offsets o = narrow_offsets_dup(lane, Bp);
 #pragma unroll
-            for (int i = 0; i < I; ++i)
+            for (int i = 0; i < I; ++i) {
                 if (warp + NW * i < nvalid)
                     racc[i] = __fadd_rn(racc[i], __fmul_rn(rar[i], lookup_row_narrow(w[i], o.w, tb, Bp >> 2)));
+                if (more) load_item(i, nd);
+            }
         }
-        if (vi + 2 < n_v) load_panel(w, rar, s_ring[(vi + 2) % kDescRing]);
     };
 #pragma unroll 1
     for (int vi = 0; vi < n_v; vi += 2) {
-        panel(std::integral_constant<int, 0>{}, vi, wA, rarA);
-        if (vi + 1 < n_v) panel(std::integral_constant<int, 1>{}, vi + 1, wB, rarB);
+        panel(std::integral_constant<int, 0>{}, vi);
+        if (vi + 1 < n_v) panel(std::integral_constant<int, 1>{}, vi + 1);
     }
 
     // ---- 3. the cluster's row partials, summed by their owner in rank order
@@ -1066,82 +773,28 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_kernel(const __gr
     if (independent) griddep_wait();   // complete only after the previous kernel
 }
 
-// ---- The batched kernel: one weight pass for up to 16 tokens -------------
+// ---- The batched kernel: one weight pass for the tokens of a pass -------
 //
 // Several activation vectors share each weight word: a CTA loads a panel's
-// words for its rows into registers once (two register sets, the panel after
-// next loading while the current one is used) and applies them to the
-// tables of every token of its pass, two tokens at a time.  The two tokens'
-// tables share each 256-byte row: entry b of byte group q is at b*256 + 4q
-// for the first token and at b*256 + 128 + 4q for the second, so both
-// lookups of a weight byte use one address (the second at a constant +128),
-// and the column offset stays below 128 (the sign-replicating byte select of
-// the address needs that).  Per token, every sum is formed in exactly the
-// order the batch-1 kernels use, and the per-token row partials are kept in
-// shared memory (any number of tokens per pass).
+// words for its rows into registers once (stream_kernel's two register sets,
+// the panel after next loading while the current one is used) and applies
+// them to every token of its pass in turn.  Each token is one step of
+// stream_kernel's panel loop -- z, the 256-entry byte tables, the lookups --
+// with the tables double-buffered across consecutive steps; a pass holds an
+// even number of tokens, so a step's buffer is its token's parity (a
+// compile-time constant, as in stream_kernel).  Per token, every sum is
+// formed in exactly stream_kernel's order; the per-token row partials live
+// in shared memory.
 //
-// Shared memory: two table buffers of 64 KB (after the last lookups, the
-// same bytes receive the cluster's row partials) | z of two steps (2
-// tokens x 256 columns each) | row partials [tp][R].
-constexpr int kBatchWarps = 16;
+// Shared memory: tables (two interleaved buffers, 64 KB; after the last
+// lookups the same bytes receive the cluster's row partials) | z of two
+// steps | row partials [tp][R].  8 warps; with 8 tokens per pass two CTAs
+// share an SM.
+constexpr int kBatchWarps = 8;
 constexpr int kMaxTokensPerPass = 16;
-constexpr int kPairTableBytes = 65536;
-
-// The two tokens' sums of the entries selected by one row's stored bytes,
-// each in lookup_row's order: eight chains (accumulator k = (2m + j/2) & 3,
-// half j & 1), then per token (lo + hi) of each k, then (k0 + k1) + (k2 + k3).
-// (nwords < 8: a narrow panel, only its first nwords stored words.)
-__device__ __forceinline__ void lookup_row_t2(const uint32_t (&w)[8], const uint32_t (&offp)[8], const float *tbl,
-                                              float &s0, float &s1, int nwords = 8) {
-    unsigned long long acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        if (m >= nwords) break;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t off = prmt(w[m], offp[m], addr_sel(jj));
-            const unsigned long long v = f2pack(lds(tbl, off), lds(tbl + 32, off));
-            const int slot = 2 * ((2 * m + (jj >> 1)) & 3) + (jj & 1);
-            acc[slot] = fadd2(acc[slot], v);
-        }
-    }
-    const unsigned long long p0 = fadd2(acc[0], acc[1]), p1 = fadd2(acc[2], acc[3]);
-    const unsigned long long p2 = fadd2(acc[4], acc[5]), p3 = fadd2(acc[6], acc[7]);
-    const unsigned long long r = fadd2(fadd2(p0, p1), fadd2(p2, p3));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(s0), "=f"(s1) : "l"(r));
-}
-
-// LUT-BSF for one panel and two tokens, built by the whole CTA (16 warps):
-// lane q builds byte group q, warp w the entries b = 16w .. 16w + 15 of both
-// tokens (z of token t at zp + 256t); entry b = T_lo[b & 15] + T_hi[b >> 4]
-// per token, as build_byte_table; token t's entries at +128t in each row.
-__device__ __forceinline__ void build_pair_table(const float *zp, float *T, int warp, int lane) {
-    float lo0[16], lo1[16];
-    {
-        const float4 za = *reinterpret_cast<const float4 *>(zp + 8 * lane);
-        sums16(za.x, za.y, za.z, za.w, lo0);
-        const float4 zc = *reinterpret_cast<const float4 *>(zp + kPanelCols + 8 * lane);
-        sums16(zc.x, zc.y, zc.z, zc.w, lo1);
-    }
-    const int h = warp;   // the high nibble of this warp's entries
-    const float4 zb = *reinterpret_cast<const float4 *>(zp + 8 * lane + 4);
-    const float4 zd = *reinterpret_cast<const float4 *>(zp + kPanelCols + 8 * lane + 4);
-    const float hi0 = __fadd_rn(__fadd_rn((h & 1) ? zb.x : -zb.x, (h & 2) ? zb.y : -zb.y),
-                                __fadd_rn((h & 4) ? zb.z : -zb.z, (h & 8) ? zb.w : -zb.w));
-    const float hi1 = __fadd_rn(__fadd_rn((h & 1) ? zd.x : -zd.x, (h & 2) ? zd.y : -zd.y),
-                                __fadd_rn((h & 4) ? zd.z : -zd.z, (h & 8) ? zd.w : -zd.w));
-    float *col = T + (16 * h) * 64 + lane;
-#pragma unroll
-    for (int v = 0; v < 16; ++v) {
-        col[v * 64] = __fadd_rn(lo0[v], hi0);
-        col[v * 64 + 32] = __fadd_rn(lo1[v], hi1);
-    }
-}
 
 template <int XT, int I>
-__global__ void __launch_bounds__(kBatchWarps * 32, 1) batched_kernel(const __grid_constant__ GemvArgs args) {
+__global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __grid_constant__ GemvArgs args) {
     constexpr int NW = kBatchWarps, NT = NW * 32;
     extern __shared__ __align__(128) float smem_f[];
     __shared__ __align__(16) GemvArgs s_args;
@@ -1160,12 +813,12 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 1) batched_kernel(const __gr
     const int nvalid = min(cpb, a.nchunks - c_first);
     const bool independent = (a.flags & FB_GEMV_INDEPENDENT) != 0;
     const int TP = a.tp, t_base = (int)blockIdx.z * TP, nt = min(TP, a.batch - t_base);
-    const int npairs = (nt + 1) >> 1, S = n_v * npairs;
+    const int S = n_v * TP;   // steps (panel, token), token fastest
 
-    float *tables = smem_f;                                   // 2 x 64 KB
-    float *zbuf = smem_f + 2 * kPairTableBytes / 4;           // [2][2][256]
-    float *accs = zbuf + 4 * kPanelCols;                      // [TP][R]
-    float *inbox = tables;                                    // after the last lookups
+    float *tables = smem_f;
+    float *zbuf = smem_f + kTableBytes / 4;
+    float *accs = zbuf + kZBytes / 4;   // [TP][R]
+    float *inbox = tables;              // after the last lookups
 
     griddep_launch_dependents();
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -1198,75 +851,96 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 1) batched_kernel(const __gr
             }
         }
     };
-    // z staging: thread t stages column t & 255 of token 2*pair + (t >> 8)
-    struct Staged {
-        float ac;
-        uint32_t x;
-        int xi;
-    };
     Staged st[2] = {{0.0f, 0u, -1}, {0.0f, 0u, -1}};
-    const int col = tid & (kPanelCols - 1), half = tid >> 8;
-    auto stage = [&](Staged &t, const PanelDesc &d, int pair, bool read_x) {
-        t.x = 0;
-        const int tok = 2 * pair + half;
-        column_source<true>(a, d, col, t.ac, t.xi);
-        if (tok >= nt) t.xi = -1;
-        if (read_x && t.xi >= 0) t.x = load_x_bits<XT>(a.x, (size_t)(t_base + tok) * a.ldx + t.xi);
+    int st_tok[2] = {0, 0};   // the token each staged set belongs to
+    // column tid of a step's panel, for token tok of the pass (none past nt)
+    auto stage = [&](int q, const PanelDesc &d, int tok, bool read_x) {
+        st_tok[q] = tok;
+        if (tok >= nt) {
+            st[q].ac = 0.0f;
+            st[q].x = 0;
+            st[q].xi = -1;
+            return;
+        }
+        stage_column<XT, true>(a, d, tid, (size_t)(t_base + tok) * a.ldx, read_x, st[q]);
     };
+    auto resolve = [&](int q) { resolve_column<XT>(a, (size_t)(t_base + st_tok[q]) * a.ldx, st[q]); };
     auto z_of = [&](const Staged &t) { return t.xi >= 0 ? __fmul_rn(t.ac, x_value<XT>(t.x)) : 0.0f; };
-    auto desc_of_step = [&](int s2) -> const PanelDesc & { return s_ring[(s2 / npairs) % kDescRing]; };
 
+    PanelDesc d0, d1;
     if (n_v > 0) {
-        const PanelDesc d0 = panel_desc(a, vb);
+        d0 = panel_desc(a, vb);
         load_panel(wA, rarA, d0);
-        stage(st[0], d0, 0, independent);
+        stage(0, d0, 0, independent);
     }
-    if (n_v > 1) load_panel(wB, rarB, panel_desc(a, vb + 1));
+    if (n_v > 1) {
+        d1 = panel_desc(a, vb + 1);
+        load_panel(wB, rarB, d1);
+    }
     if (!independent) {
         griddep_wait();
-        if (st[0].xi >= 0) st[0].x = load_x_bits<XT>(a.x, (size_t)(t_base + half) * a.ldx + st[0].xi);
+        if (st[0].xi >= 0) st[0].x = load_x_bits<XT>(a.x, (size_t)t_base * a.ldx + st[0].xi);
     }
-    zbuf[tid] = z_of(st[0]);   // step 0 -> z buffer 0
-    __syncthreads();
-    if (S > 1) stage(st[1], desc_of_step(1), 1 % npairs, true);
-    if (S > 2) stage(st[0], desc_of_step(2), 2 % npairs, true);
+    if (S > 1) stage(1, d0, 1, true);   // step 1: panel 0 (a pass holds at least two tokens)
+    resolve(0);
+    if (S > 1) resolve(1);
+    zbuf[tid] = z_of(st[0]);
+    __syncthreads();   // z of step 0, the first descriptors and the zeroed partials written
+    if (S > 2) stage(0, TP > 2 ? d0 : d1, 2 % TP, true);
 
     uint32_t off_full[8];
     full_offsets(lane, off_full);
 
-    // One step s (panel vi, token pair tp): tables of both tokens into buffer
-    // s & 1, z of step s + 1 into the other z buffer, then lookups.
-    auto panel = [&](int vi, uint32_t (&w)[I][8], float (&rar)[I]) {
+    // One step: token tok of panel vi, tables in buffer `buf` (= tok & 1).
+    auto step = [&](auto bufc, int vi, int tok, uint32_t (&w)[I][8], const float (&rar)[I]) {
+        constexpr int buf = decltype(bufc)::value;
+        const int s2 = vi * TP + tok;
         const int Bp = desc_bp(s_ring[vi % kDescRing]);
-        uint32_t offn[8];
-        if (Bp != 32) {
+        float *tb = tables + 32 * buf;
+        if (tok < nt) build_byte_table<NW>(zbuf + buf * kPanelCols, tb, warp, lane);
+        if (s2 + 1 < S) zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
+        if (s2 + 3 < S) {
+            const int s3 = s2 + 3, v3 = s3 / TP;
+            stage(buf ^ 1, s_ring[v3 % kDescRing], s3 - v3 * TP, true);
+        }
+        if (s2 + 2 < S) resolve(buf);   // step s2 + 2, staged one step ago
+        if (tid == 0 && tok == 0 && vi + 4 < n_v) s_ring[(vi + 4) % kDescRing] = panel_desc(a, vb + vi + 4);
+        __syncthreads();   // tables of this step complete; every warp done with the previous step
+        if (tok >= nt) return;
+        float *acc_t = accs + tok * R;
+        if (Bp == 32) {
+#pragma unroll
+            for (int i = 0; i < I; i += 2) {
+                const int c0 = warp + NW * i;
+                if (i + 1 < I && c0 + NW < nvalid) {
+                    float s0, s1;
+                    lookup_rows2(w[i], w[i + 1], off_full, tb, s0, s1);
+                    float *p0 = acc_t + c0 * kChunkRows + lane;
+                    *p0 = __fadd_rn(*p0, __fmul_rn(rar[i], s0));
+                    float *p1 = p0 + NW * kChunkRows;
+                    *p1 = __fadd_rn(*p1, __fmul_rn(rar[i + 1], s1));
+                } else if (c0 < nvalid) {
+                    float *p0 = acc_t + c0 * kChunkRows + lane;
+                    *p0 = __fadd_rn(*p0, __fmul_rn(rar[i], lookup_row(w[i], off_full, tb)));
+                }
+            }
+        } else {
             const Offsets o = narrow_offsets_dup(lane, Bp);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) offn[m] = o.w[m];
-        }
-#pragma unroll 1
-        for (int tp = 0; tp < npairs; ++tp) {
-            const int s2 = vi * npairs + tp, buf = s2 & 1;
-            float *tb = tables + buf * (kPairTableBytes / 4);
-            build_pair_table(zbuf + buf * 2 * kPanelCols, tb, warp, lane);
-            if (s2 + 1 < S) zbuf[(buf ^ 1) * 2 * kPanelCols + tid] = z_of(st[(s2 + 1) & 1]);
-            if (s2 + 3 < S) stage(st[(s2 + 3) & 1], desc_of_step(s2 + 3), (s2 + 3) % npairs, true);
-            if (tid == 0 && tp == 0 && vi + 4 < n_v) s_ring[(vi + 4) % kDescRing] = panel_desc(a, vb + vi + 4);
-            __syncthreads();   // tables of step s2 complete; every warp done with step s2 - 1
-#pragma unroll
             for (int i = 0; i < I; ++i) {
-                const int cl = warp + NW * i;
-                if (cl >= nvalid) continue;
-                float s0, s1;
-                if (Bp == 32)
-                    lookup_row_t2(w[i], off_full, tb, s0, s1);
-                else
-                    lookup_row_t2(w[i], offn, tb, s0, s1, Bp >> 2);
-                const int r = cl * kChunkRows + lane;
-                float *p0 = accs + (2 * tp) * R + r;
-                *p0 = __fadd_rn(*p0, __fmul_rn(rar[i], s0));
-                if (2 * tp + 1 < nt) p0[R] = __fadd_rn(p0[R], __fmul_rn(rar[i], s1));
+                const int c0 = warp + NW * i;
+                if (c0 < nvalid) {
+                    float *p0 = acc_t + c0 * kChunkRows + lane;
+                    *p0 = __fadd_rn(*p0, __fmul_rn(rar[i], lookup_row_narrow(w[i], o.w, tb, Bp >> 2)));
+                }
             }
+        }
+    };
+    auto panel = [&](int vi, uint32_t (&w)[I][8], float (&rar)[I]) {
+#pragma unroll 1
+        for (int tok = 0; tok < TP; tok += 2) {
+            step(std::integral_constant<int, 0>{}, vi, tok, w, rar);
+            step(std::integral_constant<int, 1>{}, vi, tok + 1, w, rar);
         }
         if (vi + 2 < n_v) load_panel(w, rar, s_ring[(vi + 2) % kDescRing]);
     };
@@ -1302,25 +976,24 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 1) batched_kernel(const __gr
 
 using KernelFn = void (*)(GemvArgs);
 
-template <int NW>
-KernelFn pick_xt(fb_dtype t) {
-    return t == FB_F32 ? gemv_kernel<FB_F32, NW> : t == FB_F16 ? gemv_kernel<FB_F16, NW> : gemv_kernel<FB_BF16, NW>;
-}
-
-KernelFn pick_kernel(fb_dtype t, int nw) { return nw == 16 ? pick_xt<16>(t) : pick_xt<8>(t); }
-
 template <int I>
 KernelFn pick_batched_xt(fb_dtype t) {
     return t == FB_F32 ? batched_kernel<FB_F32, I> : t == FB_F16 ? batched_kernel<FB_F16, I> : batched_kernel<FB_BF16, I>;
 }
-KernelFn pick_batched(fb_dtype t, int items) { return items == 1 ? pick_batched_xt<1>(t) : pick_batched_xt<2>(t); }
-
-template <int I>
-KernelFn pick_stream_xt(fb_dtype t) {
-    return t == FB_F32 ? stream_kernel<FB_F32, I> : t == FB_F16 ? stream_kernel<FB_F16, I> : stream_kernel<FB_BF16, I>;
+KernelFn pick_batched(fb_dtype t, int items) {
+    return items == 1 ? pick_batched_xt<1>(t) : items == 2 ? pick_batched_xt<2>(t) : pick_batched_xt<4>(t);
 }
-KernelFn pick_stream(fb_dtype t, int items) {
-    return items == 1 ? pick_stream_xt<1>(t) : items == 2 ? pick_stream_xt<2>(t) : pick_stream_xt<4>(t);
+
+template <int NW, int I>
+KernelFn pick_stream_xt(fb_dtype t) {
+    return t == FB_F32 ? stream_kernel<FB_F32, NW, I> : t == FB_F16 ? stream_kernel<FB_F16, NW, I>
+                                                                    : stream_kernel<FB_BF16, NW, I>;
+}
+KernelFn pick_stream(fb_dtype t, int nw, int items) {
+    if (nw == 16) return items == 1 ? pick_stream_xt<16, 1>(t) : items == 2 ? pick_stream_xt<16, 2>(t)
+                                                                             : pick_stream_xt<16, 4>(t);
+    return items == 1 ? pick_stream_xt<8, 1>(t) : items == 2 ? pick_stream_xt<8, 2>(t)
+                      : items == 4 ? pick_stream_xt<8, 4>(t) : pick_stream_xt<8, 8>(t);
 }
 
 fb_status check_weights(const fb_weights *W) {
@@ -1342,7 +1015,7 @@ fb_status check_weights(const fb_weights *W) {
 struct Plan {
     int M_pad, Pg, Ps, nS_pad, V, nchunks;
     int C, cpb, RB, nwarps;
-    int kind;    // 0: gemv_kernel (weights through shared-memory slots); 1: stream_kernel; 2: batched_kernel
+    int kind;    // 1: stream_kernel; 2: batched_kernel
     int items;   // stream / batched kernel: chunks per warp per panel
     int tp, passes;   // batched kernel: tokens per pass, passes (grid.z)
     int vsplit[kMaxCluster + 1];
@@ -1351,18 +1024,12 @@ struct Plan {
 
 struct PlanKey {
     int M, N, K, g, nS, Ks, batch, sms, G;
-    bool independent, slots;
+    bool independent;
     bool operator==(const PlanKey &o) const {
         return M == o.M && N == o.N && K == o.K && g == o.g && nS == o.nS && Ks == o.Ks && batch == o.batch &&
-               sms == o.sms && G == o.G && independent == o.independent && slots == o.slots;
+               sms == o.sms && G == o.G && independent == o.independent;
     }
 };
-
-void split_panels(int V, int C, int *vsplit, int *max_n) {
-    *max_n = 0;
-    for (int jj = 0; jj <= C; ++jj) vsplit[jj] = (int)((long)V * jj / C);
-    for (int jj = 0; jj < C; ++jj) *max_n = std::max(*max_n, vsplit[jj + 1] - vsplit[jj]);
-}
 
 // Byte groups a CTA looks up per row in each virtual panel (global panels of
 // base 0, 1, ..., then salient ones): 32 for a full panel and for every
@@ -1441,23 +1108,13 @@ double split_weighted(const std::vector<int> &groups, int C, int cpb, int *vspli
     return worst;
 }
 
-// Dynamic shared memory of a CTA with cpb chunks of rows and KB bases:
-// tables, z, rings, row scales, row partials and the inbox of row partials
-// pushed by the cluster (C * ceil(R / C) <= R + C floats).
-size_t smem_for(int cpb, int KB, int nv, int nw) {
-    const size_t R = (size_t)cpb * kChunkRows;
-    const int slots = nw == 16 ? Shape<16>::kSlots : Shape<8>::kSlots;
-    return (size_t)kTableBytes + kZBytes + (size_t)slots * cpb * 1024 + R * KB * 4 + R * 4 +
-           ((R + kMaxCluster + 1) & ~(size_t)1) * 4 + (size_t)nv * sizeof(PanelDesc);
-}
-
 // Dynamic shared memory of a stream_kernel CTA with cpb chunks of rows:
 // tables, z of two panels, the cluster inbox (C * ceil(R / C) <= R + C floats).
 size_t stream_smem(int cpb) {
     return (size_t)kTableBytes + kZBytes + (size_t)((cpb * kChunkRows + kMaxCluster + 1) & ~1) * 4;
 }
 
-int stream_items(int cpb) { return cpb <= kStreamWarps ? 1 : cpb <= 2 * kStreamWarps ? 2 : 4; }
+int stream_items(int cpb, int nw = kStreamWarps) { return cpb <= nw ? 1 : cpb <= 2 * nw ? 2 : cpb <= 4 * nw ? 4 : 8; }
 
 // Plan of the streaming kernel (8 warps, two CTAs per SM, up to 4 chunks per
 // warp, clusters of up to 16 CTAs).
@@ -1478,7 +1135,7 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
     pl.nchunks = pl.M_pad / kChunkRows;
     pl.nwarps = kStreamWarps;
     pl.kind = 1;
-    const int max_cpb = 4 * kStreamWarps;
+    const int max_cpb = 4 * kStreamWarps;   // default plans: up to 4 items per warp
     auto set = [&](int C, int cpb) {
         pl.C = std::min(C, pl.V);
         pl.cpb = std::min(cpb, pl.nchunks);
@@ -1515,20 +1172,23 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         }
     }
     if (const char *ov = getenv("FB_PLAN")) {
-        int oc = 0, ocpb = 0;
-        if (sscanf(ov, "%d,%d", &oc, &ocpb) == 2 && oc >= 1 && ocpb >= 1)
-            set(std::min(oc, kMaxCluster), std::min(ocpb, max_cpb));
+        int oc = 0, ocpb = 0, onw = 0;
+        if (sscanf(ov, "%d,%d,%d", &oc, &ocpb, &onw) >= 2 && oc >= 1 && ocpb >= 1) {
+            if (onw == 16) pl.nwarps = 16;
+            set(std::min(oc, kMaxCluster), std::min(ocpb, pl.nwarps == 16 ? 4 * 16 : 8 * kStreamWarps));
+        }
     }
-    pl.items = stream_items(pl.cpb);
+    pl.items = stream_items(pl.cpb, pl.nwarps);
     pl.smem = stream_smem(pl.cpb);
     return pl;
 }
 
-// Plan of the batched kernel (16 warps, one CTA per SM): row blocks of up
-// to 32 chunks (two per warp), up to 16 tokens per pass, and as many CTAs
-// per cluster (up to 16) as fill the SMs once.
+// Plan of the batched kernel (8 warps): row blocks of up to 32 chunks, an
+// even number of tokens per pass (8 by default: two CTAs share an SM; 16
+// with FB_PLAN's third field), and as many CTAs per cluster (up to 16) as
+// fill the SMs twice.
 size_t batched_smem(int cpb, int tp) {
-    return (size_t)2 * kPairTableBytes + 4 * kPanelCols * 4 + (size_t)tp * cpb * kChunkRows * 4;
+    return (size_t)kTableBytes + kZBytes + (size_t)tp * cpb * kChunkRows * 4;
 }
 
 Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
@@ -1537,29 +1197,37 @@ Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
     pl.Pg = num_panels(W->N);
     pl.nS_pad = W->nS > 0 ? round_up(W->nS, 32) : 0;
     pl.Ps = W->nS > 0 ? num_panels(pl.nS_pad) : 0;
-    pl.V = pl.Pg * W->K + pl.Ps * (W->nS > 0 ? W->Ks : 0);
+    const std::vector<int> groups = vpanel_groups(W->N, W->K, 0, pl.nS_pad, W->nS > 0 ? W->Ks : 0);
+    pl.V = (int)groups.size();
     pl.nchunks = pl.M_pad / kChunkRows;
     pl.nwarps = kBatchWarps;
     pl.kind = 2;
-    pl.tp = std::min(batch, kMaxTokensPerPass);
+    int tp_max = 8, oc = 0, ocpb = 0, otp = 0;
+    const char *ov = getenv("FB_PLAN");
+    if (ov && sscanf(ov, "%d,%d,%d", &oc, &ocpb, &otp) >= 2 && otp >= 2) tp_max = std::min(otp, kMaxTokensPerPass);
+    tp_max &= ~1;
+    pl.tp = std::min(round_up(batch, 2), tp_max);
     pl.passes = ceil_div(batch, pl.tp);
-    const int max_cpb = 2 * kBatchWarps;
+    const int max_cpb = 4 * kBatchWarps;
     pl.RB = ceil_div(pl.nchunks, max_cpb);
     pl.cpb = ceil_div(pl.nchunks, pl.RB);
     const long blocks = (long)pl.RB * pl.passes;
-    int C = blocks >= sms ? 1 : (int)(sms / blocks);
+    int C = blocks >= 2L * sms ? 1 : (int)(2L * sms / blocks);
     C = std::max(1, std::min(std::min(C, kMaxCluster), pl.V));
-    if (const char *ov = getenv("FB_PLAN")) {
-        int oc = 0, ocpb = 0;
-        if (sscanf(ov, "%d,%d", &oc, &ocpb) == 2 && oc >= 1 && ocpb >= 1) {
-            C = std::min(std::min(oc, kMaxCluster), pl.V);
-            pl.cpb = std::min(std::min(ocpb, max_cpb), pl.nchunks);
-            pl.RB = ceil_div(pl.nchunks, pl.cpb);
-        }
+    if (ov && oc >= 1 && ocpb >= 1) {
+        C = std::min(std::min(oc, kMaxCluster), pl.V);
+        pl.cpb = std::min(std::min(ocpb, max_cpb), pl.nchunks);
+        pl.RB = ceil_div(pl.nchunks, pl.cpb);
+    }
+    // the cluster's partials for every token of the pass are received in the
+    // table bytes: C * tp * ceil(R / C) <= tp * (R + C) floats must fit
+    while (pl.cpb > 1 && (size_t)pl.tp * (pl.cpb * kChunkRows + kMaxCluster) * 4 > (size_t)kTableBytes) {
+        --pl.cpb;
+        pl.RB = ceil_div(pl.nchunks, pl.cpb);
     }
     pl.C = C;
-    split_weighted(vpanel_groups(W->N, W->K, 0, pl.nS_pad, W->nS > 0 ? W->Ks : 0), pl.C, pl.cpb, pl.vsplit);
-    pl.items = pl.cpb <= kBatchWarps ? 1 : 2;
+    split_weighted(groups, pl.C, pl.cpb, pl.vsplit);
+    pl.items = stream_items(pl.cpb);
     pl.smem = batched_smem(pl.cpb, pl.tp);
     return pl;
 }
@@ -1575,113 +1243,29 @@ Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
 //    barrier, lookups), times the number of waves; more CTAs per cluster
 //    shorten a CTA's panel list.
 // Both rules were fitted to timings of this kernel on B200.
-Plan make_plan(const fb_weights *W, int batch, int sms, bool independent, bool slots, int G) {
-    if (G > 0 || !slots) {
-        if (batch > 1) return make_batched_plan(W, batch, sms);
-        Plan pl = make_stream_plan(W, batch, sms, independent, G);
-        pl.tp = 1;
-        pl.passes = 1;
-        return pl;
-    }
-    Plan pl;
-    pl.kind = 0;
-    pl.items = 2;
+// The launch plan of a call: the batched kernel for more than one token,
+// else the streaming kernel.
+Plan make_plan(const fb_weights *W, int batch, int sms, bool independent, int G) {
+    if (batch > 1) return make_batched_plan(W, batch, sms);
+    Plan pl = make_stream_plan(W, batch, sms, independent, G);
     pl.tp = 1;
-    pl.passes = batch;
-    pl.M_pad = round_up(W->M, kChunkRows);
-    pl.Pg = num_panels(W->N);
-    pl.nS_pad = W->nS > 0 ? round_up(W->nS, 32) : 0;
-    pl.Ps = W->nS > 0 ? num_panels(pl.nS_pad) : 0;
-    pl.V = pl.Pg * W->K + pl.Ps * (W->nS > 0 ? W->Ks : 0);
-    pl.nchunks = pl.M_pad / kChunkRows;
-    const int nw = independent ? 16 : 8, max_cpb = 2 * nw;   // the CTA shape (Shape<NW>)
-    pl.nwarps = nw;
-    const int KB = W->K + (W->nS > 0 ? W->Ks : 0);
-    const int occ_regs = 65536 / (nw * 32 * 128);   // CTAs per SM by registers (128 per thread)
-    auto fits = [&](int C, int cpb) {
-        int vs[kMaxCluster + 1], nvm;
-        split_panels(pl.V, C, vs, &nvm);
-        return smem_for(cpb, KB, nvm, nw) <= kMaxDynSmem;
-    };
-    auto set = [&](int C, int cpb) {
-        pl.C = C;
-        pl.RB = ceil_div(pl.nchunks, cpb);
-        // independent plans balance the row blocks (the same rows, less padding)
-        pl.cpb = independent ? ceil_div(pl.nchunks, pl.RB) : cpb;
-        int nvm;
-        split_panels(pl.V, C, pl.vsplit, &nvm);
-    };
-    if (independent) {
-        int cpb = std::min(max_cpb, pl.nchunks);
-        while (cpb > 1 && !fits(2, cpb)) --cpb;
-        const int RB = ceil_div(pl.nchunks, cpb);
-        set(std::min(pl.V, RB <= 8 ? 2 : 1), cpb);
-    } else {
-        const double fixed = 4.0, per_panel = 1.2, per_item = 0.1;   // microseconds
-        double best = 1e300;
-        set(1, std::min(max_cpb, pl.nchunks));
-        for (int C = 1; C <= std::min(kMaxSlotCluster, pl.V); ++C) {
-            int vs[kMaxCluster + 1], nvm;
-            split_panels(pl.V, C, vs, &nvm);
-            // whole chunks per warp (uneven splits measured slower on B200), or
-            // the whole matrix when it has fewer chunks than warps
-            for (int cpb = std::min(nw, pl.nchunks); cpb <= std::min(max_cpb, pl.nchunks);
-                 cpb += (pl.nchunks < nw ? max_cpb : nw)) {
-                const int RB = ceil_div(pl.nchunks, cpb);
-                if (RB > 65535) continue;
-                const size_t smem = smem_for(cpb, KB, nvm, nw);
-                if (smem > kMaxDynSmem) continue;
-                const int occ = std::max(1, std::min(occ_regs, (int)(kSmemPerSM / (smem + kStaticSmem + 1024))));
-                const long ctas = (long)C * RB * batch;
-                const double waves = std::ceil((double)ctas / ((double)sms * occ));
-                const double cost = waves * (fixed + nvm * (per_panel + std::ceil((double)cpb / nw) * per_item));
-                if (cost < best * 0.999) {
-                    best = cost;
-                    set(C, cpb);
-                }
-            }
-        }
-    }
-    // Tuning aid: FB_PLAN="C,cpb" forces the cluster size and row block
-    // (clamped to what the matrix allows); read at each plan construction.
-    if (const char *ov = getenv("FB_PLAN")) {
-        int oc = 0, ocpb = 0;
-        if (sscanf(ov, "%d,%d", &oc, &ocpb) == 2 && oc >= 1 && ocpb >= 1) {
-            pl.C = std::min(std::min(oc, kMaxSlotCluster), pl.V);
-            pl.cpb = std::min(std::min(ocpb, max_cpb), pl.nchunks);
-            int nvm;
-            split_panels(pl.V, pl.C, pl.vsplit, &nvm);
-            while (pl.cpb > 1 && smem_for(pl.cpb, KB, nvm, nw) > kMaxDynSmem) --pl.cpb;
-            pl.RB = ceil_div(pl.nchunks, pl.cpb);
-        }
-    }
-    int nv_max = 0;
-    for (int jj = 0; jj < pl.C; ++jj) nv_max = std::max(nv_max, pl.vsplit[jj + 1] - pl.vsplit[jj]);
-    pl.smem = smem_for(pl.cpb, KB, nv_max, nw);
+    pl.passes = 1;
     return pl;
 }
 
-// Which kernel a call runs: the streaming kernel, except for the test mode
-// of the weight-copy waits (only the slot kernel copies weights and waits).
-bool use_slots(unsigned flags) {
-    (void)flags;
-    const char *k = getenv("FB_KERNEL");
-    return k && k[0] == 's' && k[1] == 'l';
-}
-
-const Plan &cached_plan(const fb_weights *W, int batch, int sms, bool independent, bool slots, int G = 0) {
+const Plan &cached_plan(const fb_weights *W, int batch, int sms, bool independent, int G = 0) {
     struct Entry {
         PlanKey key;
         Plan plan;
     };
     thread_local Entry memo[16];
     thread_local int used = 0, next = 0;
-    const PlanKey key{W->M, W->N, W->K, W->g, W->nS, W->nS > 0 ? W->Ks : 0, batch, sms, G, independent, slots};
+    const PlanKey key{W->M, W->N, W->K, W->g, W->nS, W->nS > 0 ? W->Ks : 0, batch, sms, G, independent};
     for (int i = 0; i < used; ++i)
         if (memo[i].key == key) return memo[i].plan;
     Entry &e = memo[next];
     e.key = key;
-    e.plan = make_plan(W, batch, sms, independent, slots, G);
+    e.plan = make_plan(W, batch, sms, independent, G);
     next = (next + 1) % 16;
     used = std::min(used + 1, 16);
     return e.plan;
@@ -1760,9 +1344,9 @@ static fb_status launch_gemv(const fb_weights *const *Ws, int n, const void *X, 
     // the plan of the largest matrix (the format, hence the panels, is shared)
     fb_weights Wp = *W;
     Wp.M = M_max;
-    const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0, use_slots(flags), G);
-    const KernelFn fn = pl.kind == 0 ? pick_kernel(t, pl.nwarps)
-                        : pl.kind == 1 ? pick_stream(t, pl.items) : pick_batched(t, pl.items);
+    const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0, G);
+    if (pl.smem > kMaxDynSmem) return FB_ERR_UNSUPPORTED;   // (no plan asks for more; a guard)
+    const KernelFn fn = pl.kind == 1 ? pick_stream(t, pl.nwarps, pl.items) : pick_batched(t, pl.items);
     if (!prepare_kernel(fn, pl.smem)) return FB_ERR_CUDA;
 
     GemvArgs a;
@@ -1877,7 +1461,7 @@ extern "C" fb_status fb_gemv_grouped(const fb_weights *const *W, int n, const vo
 extern "C" fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned flags, int sms, int *out) {
     if (check_weights(W) != FB_OK || batch < 1 || batch > kMaxBatch || sms < 1 || !out || (flags & ~kKnownFlags))
         return FB_ERR_INVALID_VALUE;
-    const Plan &pl = cached_plan(W, batch, sms, (flags & FB_GEMV_INDEPENDENT) != 0, use_slots(flags));
+    const Plan &pl = cached_plan(W, batch, sms, (flags & FB_GEMV_INDEPENDENT) != 0);
     out[0] = pl.C;
     out[1] = pl.cpb;
     out[2] = pl.RB;
