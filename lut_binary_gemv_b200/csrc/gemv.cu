@@ -826,28 +826,26 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
     for (int i = tid; i < TP * R; i += NT) accs[i] = 0.0f;
     if (tid < kDescRing - 4 && tid < n_v) s_ring[tid] = panel_desc(a, vb + tid);
 
-    uint32_t wA[I][8], wB[I][8];
-    float rarA[I], rarB[I];
-    auto load_panel = [&](uint32_t (&w)[I][8], float (&rar)[I], const PanelDesc &d) {
+    // One weight register set, as in stream_kernel: an item's registers take
+    // the next panel's words right after the pass's last token used them.
+    uint32_t w[I][8];
+    float rar[I];
+    auto load_item = [&](int i, const PanelDesc &d) {
         const int Bp = desc_bp(d);
         const size_t blk = 32u * (unsigned)Bp;
-        const float *src = row_scales(a, d.kb);
+        const int cl = warp + NW * i;
+        const int row = (c_first + cl) * kChunkRows + lane;
+        rar[i] = cl < nvalid && row < a.M ? __ldg(row_scales(a, d.kb) + row) : 0.0f;
+        if (cl < nvalid) {
+            const uint8_t *p = d.pl + blk * (size_t)(c_first + cl);
+            if (Bp == 32) {
+                const uint4 x0 = ldg_stream(p + 16 * lane), x1 = ldg_stream(p + 512 + 16 * lane);
+                w[i][0] = x0.x; w[i][1] = x0.y; w[i][2] = x0.z; w[i][3] = x0.w;
+                w[i][4] = x1.x; w[i][5] = x1.y; w[i][6] = x1.z; w[i][7] = x1.w;
+            } else {
+                const Words r = load_item_narrow(p, Bp, lane);
 #pragma unroll
-        for (int i = 0; i < I; ++i) {
-            const int cl = warp + NW * i;
-            const int row = (c_first + cl) * kChunkRows + lane;
-            rar[i] = cl < nvalid && row < a.M ? __ldg(src + row) : 0.0f;
-            if (cl < nvalid) {
-                const uint8_t *p = d.pl + blk * (size_t)(c_first + cl);
-                if (Bp == 32) {
-                    const uint4 x0 = ldg_stream(p + 16 * lane), x1 = ldg_stream(p + 512 + 16 * lane);
-                    w[i][0] = x0.x; w[i][1] = x0.y; w[i][2] = x0.z; w[i][3] = x0.w;
-                    w[i][4] = x1.x; w[i][5] = x1.y; w[i][6] = x1.z; w[i][7] = x1.w;
-                } else {
-                    const Words r = load_item_narrow(p, Bp, lane);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) w[i][m] = r.w[m];
-                }
+                for (int m = 0; m < 8; ++m) w[i][m] = r.w[m];
             }
         }
     };
@@ -870,13 +868,11 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
     PanelDesc d0, d1;
     if (n_v > 0) {
         d0 = panel_desc(a, vb);
-        load_panel(wA, rarA, d0);
+#pragma unroll
+        for (int i = 0; i < I; ++i) load_item(i, d0);
         stage(0, d0, 0, independent);
     }
-    if (n_v > 1) {
-        d1 = panel_desc(a, vb + 1);
-        load_panel(wB, rarB, d1);
-    }
+    if (n_v > 1) d1 = panel_desc(a, vb + 1);
     if (!independent) {
         griddep_wait();
         if (st[0].xi >= 0) st[0].x = load_x_bits<XT>(a.x, (size_t)t_base * a.ldx + st[0].xi);
@@ -891,8 +887,9 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
     uint32_t off_full[8];
     full_offsets(lane, off_full);
 
-    // One step: token tok of panel vi, tables in buffer `buf` (= tok & 1).
-    auto step = [&](auto bufc, int vi, int tok, uint32_t (&w)[I][8], const float (&rar)[I]) {
+    // One step: token tok of panel vi, tables in buffer `buf` (= tok & 1);
+    // the pass's last step reloads each item with the next panel's words.
+    auto step = [&](auto bufc, int vi, int tok) {
         constexpr int buf = decltype(bufc)::value;
         const int s2 = vi * TP + tok;
         const int Bp = desc_bp(s_ring[vi % kDescRing]);
@@ -906,6 +903,9 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
         if (s2 + 2 < S) resolve(buf);   // step s2 + 2, staged one step ago
         if (tid == 0 && tok == 0 && vi + 4 < n_v) s_ring[(vi + 4) % kDescRing] = panel_desc(a, vb + vi + 4);
         __syncthreads();   // tables of this step complete; every warp done with the previous step
+        // the pass's last token with lookups: after it, the items reload
+        const bool reload = tok == min(TP, nt) - 1 && vi + 1 < n_v;
+        const PanelDesc &nd = s_ring[(vi + 1) % kDescRing];
         if (tok >= nt) return;
         float *acc_t = accs + tok * R;
         if (Bp == 32) {
@@ -923,6 +923,10 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
                     float *p0 = acc_t + c0 * kChunkRows + lane;
                     *p0 = __fadd_rn(*p0, __fmul_rn(rar[i], lookup_row(w[i], off_full, tb)));
                 }
+                if (reload) {
+                    load_item(i, nd);
+                    if (i + 1 < I) load_item(i + 1, nd);
+                }
             }
         } else {
             const Offsets o = narrow_offsets_dup(lane, Bp);
@@ -933,21 +937,17 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
                     float *p0 = acc_t + c0 * kChunkRows + lane;
                     *p0 = __fadd_rn(*p0, __fmul_rn(rar[i], lookup_row_narrow(w[i], o.w, tb, Bp >> 2)));
                 }
+                if (reload) load_item(i, nd);
             }
         }
     };
-    auto panel = [&](int vi, uint32_t (&w)[I][8], float (&rar)[I]) {
+#pragma unroll 1
+    for (int vi = 0; vi < n_v; ++vi) {
 #pragma unroll 1
         for (int tok = 0; tok < TP; tok += 2) {
-            step(std::integral_constant<int, 0>{}, vi, tok, w, rar);
-            step(std::integral_constant<int, 1>{}, vi, tok + 1, w, rar);
+            step(std::integral_constant<int, 0>{}, vi, tok);
+            step(std::integral_constant<int, 1>{}, vi, tok + 1);
         }
-        if (vi + 2 < n_v) load_panel(w, rar, s_ring[(vi + 2) % kDescRing]);
-    };
-#pragma unroll 1
-    for (int vi = 0; vi < n_v; vi += 2) {
-        panel(vi, wA, rarA);
-        if (vi + 1 < n_v) panel(vi + 1, wB, rarB);
     }
 
     // ---- the cluster's row partials, per token, in a fixed order ------------
@@ -981,7 +981,8 @@ KernelFn pick_batched_xt(fb_dtype t) {
     return t == FB_F32 ? batched_kernel<FB_F32, I> : t == FB_F16 ? batched_kernel<FB_F16, I> : batched_kernel<FB_BF16, I>;
 }
 KernelFn pick_batched(fb_dtype t, int items) {
-    return items == 1 ? pick_batched_xt<1>(t) : items == 2 ? pick_batched_xt<2>(t) : pick_batched_xt<4>(t);
+    return items == 1 ? pick_batched_xt<1>(t) : items == 2 ? pick_batched_xt<2>(t)
+                      : items == 4 ? pick_batched_xt<4>(t) : pick_batched_xt<8>(t);
 }
 
 template <int NW, int I>
@@ -1116,11 +1117,10 @@ size_t stream_smem(int cpb) {
 
 int stream_items(int cpb, int nw = kStreamWarps) { return cpb <= nw ? 1 : cpb <= 2 * nw ? 2 : cpb <= 4 * nw ? 4 : 8; }
 
-// Plan of the streaming kernel (8 warps, two CTAs per SM, up to 4 chunks per
+// Plan of the streaming kernel (8 warps, two CTAs per SM, up to 8 chunks per
 // warp, clusters of up to 16 CTAs).
 //  * Independent calls overlap their neighbours: the largest row blocks
-//    (fewest table builds per row), C = 2 for matrices of at most 8 row
-//    blocks, else 1.
+//    (64 chunks: fewest table builds per row), C = 2.
 //  * A dependent call is timed alone: latency model of a fixed cost plus,
 //    per panel a CTA works through, a table build and its lookups, times
 //    the waves; clusters beyond one CTA add a reduction.
@@ -1143,8 +1143,10 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         split_weighted(groups, pl.C, pl.cpb, pl.vsplit);
     };
     if (independent) {
-        const int RB = ceil_div(pl.nchunks, max_cpb);
-        set(RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
+        // row blocks of up to 64 chunks (eight per warp: table builds and
+        // per-panel work spread over the most rows), two CTAs per cluster
+        const int RB = ceil_div(pl.nchunks, 8 * kStreamWarps);
+        set(2, ceil_div(pl.nchunks, RB));
     } else {
         // One CTA per SM at most (the next call's CTAs take the SMs' other
         // half), minimising the largest CTA's shared-memory work (table
@@ -1208,7 +1210,7 @@ Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
     tp_max &= ~1;
     pl.tp = std::min(round_up(batch, 2), tp_max);
     pl.passes = ceil_div(batch, pl.tp);
-    const int max_cpb = 4 * kBatchWarps;
+    const int max_cpb = 4 * kBatchWarps;   // default: 4 items per warp (8 with the tuning override)
     pl.RB = ceil_div(pl.nchunks, max_cpb);
     pl.cpb = ceil_div(pl.nchunks, pl.RB);
     const long blocks = (long)pl.RB * pl.passes;
@@ -1216,7 +1218,7 @@ Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
     C = std::max(1, std::min(std::min(C, kMaxCluster), pl.V));
     if (ov && oc >= 1 && ocpb >= 1) {
         C = std::min(std::min(oc, kMaxCluster), pl.V);
-        pl.cpb = std::min(std::min(ocpb, max_cpb), pl.nchunks);
+        pl.cpb = std::min(std::min(ocpb, 2 * max_cpb), pl.nchunks);
         pl.RB = ceil_div(pl.nchunks, pl.cpb);
     }
     // the cluster's partials for every token of the pass are received in the
