@@ -1117,10 +1117,11 @@ size_t stream_smem(int cpb) {
 
 int stream_items(int cpb, int nw = kStreamWarps) { return cpb <= nw ? 1 : cpb <= 2 * nw ? 2 : cpb <= 4 * nw ? 4 : 8; }
 
-// Plan of the streaming kernel (8 warps, two CTAs per SM, up to 8 chunks per
-// warp, clusters of up to 16 CTAs).
-//  * Independent calls overlap their neighbours: the largest row blocks
-//    (64 chunks: fewest table builds per row), C = 2.
+// Plan of the streaming kernel (8 warps, two CTAs per SM, up to 4 chunks per
+// warp -- 8 with the tuning override -- and clusters of up to 16 CTAs).
+//  * Independent calls overlap their neighbours: row blocks of 32 chunks
+//    (few table builds per row), C = 2 for matrices of at most 8 row
+//    blocks, else 1.
 //  * A dependent call is timed alone: latency model of a fixed cost plus,
 //    per panel a CTA works through, a table build and its lookups, times
 //    the waves; clusters beyond one CTA add a reduction.
@@ -1143,10 +1144,12 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         split_weighted(groups, pl.C, pl.cpb, pl.vsplit);
     };
     if (independent) {
-        // row blocks of up to 64 chunks (eight per warp: table builds and
-        // per-panel work spread over the most rows), two CTAs per cluster
-        const int RB = ceil_div(pl.nchunks, 8 * kStreamWarps);
-        set(2, ceil_div(pl.nchunks, RB));
+        // row blocks of up to 32 chunks, C = 2 for matrices of at most 8 row
+        // blocks, else 1.  (64-chunk blocks run faster on one large matrix
+        // but make each CTA live so long that graphs of mixed calls, the 7B
+        // step, lose more to filling and draining than they gain.)
+        const int RB = ceil_div(pl.nchunks, max_cpb);
+        set(RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
     } else {
         // One CTA per SM at most (the next call's CTAs take the SMs' other
         // half), minimising the largest CTA's shared-memory work (table
