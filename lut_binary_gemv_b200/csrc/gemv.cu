@@ -578,6 +578,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
     __shared__ __align__(16) GemvArgs s_args;
     __shared__ __align__(16) PanelDesc s_ring[kDescRing];
     __shared__ __align__(8) unsigned long long s_inbox_bar;   // the cluster's row partials have landed
+    // The next call in the stream may launch at once: it reads nothing this
+    // kernel writes before its own programmatic-launch wait, and a call
+    // flagged independent completes only after this one.
+    griddep_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     static_assert(offsetof(GemvArgs, mats) % 4 == 0, "parameter block copied as words");
     for (int i = tid; i < (int)(offsetof(GemvArgs, mats) / 4); i += blockDim.x)
@@ -618,7 +622,6 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
     float *zbuf = smem_f + kTableBytes / 4;
     float *part = zbuf + 2 * kPanelCols;   // cluster inbox: R + C floats
 
-    griddep_launch_dependents();
     // The row partials reach their owner CTA as asynchronous remote stores
     // that complete on the owner's inbox barrier: it expects C * (its rows)
     // * 4 bytes (its own slot included).  The barrier is initialised and its
@@ -770,7 +773,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
         const int row = c_first * kChunkRows + r;
         if (row < a.M) a.y[(size_t)b * a.ldy + row] = ok ? sum : __int_as_float(0x7fc00000);
     }
-    if (independent) griddep_wait();   // complete only after the previous kernel
+    // complete only after the previous kernel: one CTA waiting is enough (the
+    // grid completes when its last CTA exits), and the others free their SM
+    // slots for the calls that follow
+    if (independent && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) griddep_wait();
 }
 
 // ---- The batched kernel: one weight pass for the tokens of a pass -------
@@ -799,6 +805,7 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
     extern __shared__ __align__(128) float smem_f[];
     __shared__ __align__(16) GemvArgs s_args;
     __shared__ __align__(16) PanelDesc s_ring[kDescRing];
+    griddep_launch_dependents();   // (as in stream_kernel)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int i = tid; i < (int)(offsetof(GemvArgs, mats) / 4); i += blockDim.x)
         reinterpret_cast<int *>(&s_args)[i] = reinterpret_cast<const int *>(&args)[i];
@@ -820,7 +827,6 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
     float *accs = zbuf + kZBytes / 4;   // [TP][R]
     float *inbox = tables;              // after the last lookups
 
-    griddep_launch_dependents();
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
     for (int i = tid; i < TP * R; i += NT) accs[i] = 0.0f;
@@ -971,7 +977,7 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
         const int row = c_first * kChunkRows + r;
         if (row < a.M) a.y[(size_t)(t_base + t) * a.ldy + row] = sum;
     }
-    if (independent) griddep_wait();
+    if (independent && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) griddep_wait();   // (as stream_kernel)
 }
 
 using KernelFn = void (*)(GemvArgs);
