@@ -1032,11 +1032,36 @@ struct Plan {
 struct PlanKey {
     int M, N, K, g, nS, Ks, batch, sms, G;
     bool independent;
+    int rows[kMaxGroup];   // a grouped call: every matrix's M (0 past the last)
     bool operator==(const PlanKey &o) const {
         return M == o.M && N == o.N && K == o.K && g == o.g && nS == o.nS && Ks == o.Ks && batch == o.batch &&
-               sms == o.sms && G == o.G && independent == o.independent;
+               sms == o.sms && G == o.G && independent == o.independent &&
+               std::equal(rows, rows + kMaxGroup, o.rows);
     }
 };
+
+// The matrices of one launch (a grouped call's row blocks follow one another
+// in the grid): their row counts.
+struct Group {
+    int n = 1;
+    int M[kMaxGroup] = {0, 0, 0, 0};
+};
+
+// Row blocks of a launch whose blocks hold cpb chunks of 32 rows.
+long group_row_blocks(const Group &grp, int cpb) {
+    long rb = 0;
+    for (int m = 0; m < grp.n; ++m) rb += ceil_div(round_up(grp.M[m], kChunkRows) / kChunkRows, cpb);
+    return rb;
+}
+
+// Clusters of C stream_kernel CTAs that can be resident at once with two
+// CTAs per SM.  A cluster stays within one GPC, so this is less than 2 * sms
+// / C; the table is cudaOccupancyMaxActiveClusters on B200 (148 SMs) for
+// such a kernel, scaled for other SM counts.
+int cluster_capacity(int sms, int C) {
+    static const int k148[kMaxCluster + 1] = {0, 296, 148, 93, 71, 56, 45, 37, 33, 30, 26, 21, 21, 17, 14, 14, 14};
+    return std::max(1, (int)((long)k148[std::min(std::max(C, 1), kMaxCluster)] * sms / 148));
+}
 
 // Byte groups a CTA looks up per row in each virtual panel (global panels of
 // base 0, 1, ..., then salient ones): 32 for a full panel and for every
@@ -1128,10 +1153,12 @@ int stream_items(int cpb, int nw = kStreamWarps) { return cpb <= nw ? 1 : cpb <=
 //  * Independent calls overlap their neighbours: row blocks of 32 chunks
 //    (few table builds per row), C = 2 for matrices of at most 8 row
 //    blocks, else 1.
-//  * A dependent call is timed alone: latency model of a fixed cost plus,
-//    per panel a CTA works through, a table build and its lookups, times
-//    the waves; clusters beyond one CTA add a reduction.
-Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent, int G) {
+//  * A call that waits for its predecessor: the plan of least modelled
+//    latency (per panel a CTA works through, a fixed cost and a cost per
+//    chunk of rows; times the waves of clusters that fit at two CTAs per
+//    SM; plus a cost per CTA of a cluster), row blocks counted over the
+//    whole launch of a grouped call.
+Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent, int G, const Group &grp) {
     Plan pl;
     pl.M_pad = round_up(W->M, kChunkRows);
     pl.Pg = num_panels(W->N);
@@ -1157,29 +1184,45 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         const int RB = ceil_div(pl.nchunks, max_cpb);
         set(RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
     } else {
-        // One CTA per SM at most (the next call's CTAs take the SMs' other
-        // half), minimising the largest CTA's shared-memory work (table
-        // builds and lookups, split_weighted) plus a cluster-reduction term.
-        // Row blocks of whole chunks per warp (8, 16, 24 or 32 chunks; the
-        // whole matrix when it has fewer than 8).
+        // Latency model of a call that waits for its predecessor (fitted to
+        // dependent chains of this kernel on B200 over the shapes 4096^2,
+        // 11008x4096, 4096x11008, 8192^2, 28672x8192, 8192x28672 and the
+        // grouped q/k/v and gate/up calls): a CTA spends about 1 us per
+        // panel on the table build, the barrier and the staging, plus 0.37
+        // us per chunk of rows each warp looks up; the call takes its
+        // slowest CTA's panels once per wave of clusters, a wave being what
+        // fits at two CTAs per SM (90% of it: the neighbouring calls hold
+        // some slots); each CTA of a cluster adds 0.2 us (the reduction, the
+        // cluster's launch).  Row blocks of whole chunks per warp (8, 16, 24
+        // or 32 chunks), clusters of 1, 2, 3, 4, 6, 8, 10, 12 or 16 CTAs.
+        static const int kClusters[] = {1, 2, 3, 4, 6, 8, 10, 12, 16};
+        int nch_max = 0;
+        for (int m = 0; m < grp.n; ++m) nch_max = std::max(nch_max, round_up(grp.M[m], kChunkRows) / kChunkRows);
         double best = 1e300;
         set(1, std::min(max_cpb, pl.nchunks));
         for (int cpb = kStreamWarps; cpb <= max_cpb; cpb += kStreamWarps) {
-            const int c = std::min(cpb, pl.nchunks);
-            const long RB = ceil_div(pl.nchunks, c);
+            const int c = std::min(cpb, nch_max);
+            const long RB = group_row_blocks(grp, c) * batch;
             if (RB > 65535) continue;
-            for (int C = 1; C <= std::min(kMaxCluster, pl.V); ++C) {
-                const long ctas = (long)C * RB * batch;
-                const double waves = std::ceil((double)ctas / sms);
+            const double per_chunk = 0.37 * std::ceil((double)c / kStreamWarps);
+            for (int C : kClusters) {
+                if (C > std::min(kMaxCluster, pl.V)) break;
                 int vs[kMaxCluster + 1];
-                const double work = split_weighted(groups, C, c, vs);
-                const double cost = waves * work + (C > 1 ? 1000.0 : 0.0);
+                split_weighted(groups, C, c, vs);
+                double slowest = 0.0;
+                for (int q = 0; q < C; ++q) {
+                    double t = 0.0;
+                    for (int v = vs[q]; v < vs[q + 1]; ++v) t += 1.0 + per_chunk * groups[v] / 32.0;
+                    slowest = std::max(slowest, t);
+                }
+                const long cap = std::max(1, (int)(0.9 * cluster_capacity(sms, C)));
+                const double cost = (double)ceil_div(RB, cap) * slowest + 0.2 * C;
                 if (cost < best * 0.999) {
                     best = cost;
                     set(C, c);
                 }
             }
-            if (c == pl.nchunks) break;
+            if (c == nch_max) break;
         }
     }
     if (const char *ov = getenv("FB_PLAN")) {
@@ -1243,40 +1286,35 @@ Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
     return pl;
 }
 
-// The launch plan: cluster size C (the split of the V virtual panels over
-// the cluster's CTAs) and row block size (cpb chunks of 32 rows).
-//  * Calls flagged independent (16-warp CTAs) overlap their neighbours, so
-//    the plan that does the least work wins: the largest row blocks (fewest
-//    table builds per row), C = 2 for matrices of at most 8 row blocks,
-//    else 1.
-//  * A dependent call (8-warp CTAs, two per SM) is timed alone: its latency
-//    is about a fixed 4 us plus 1.2 us per panel a CTA works through (build,
-//    barrier, lookups), times the number of waves; more CTAs per cluster
-//    shorten a CTA's panel list.
-// Both rules were fitted to timings of this kernel on B200.
 // The launch plan of a call: the batched kernel for more than one token,
-// else the streaming kernel.
-Plan make_plan(const fb_weights *W, int batch, int sms, bool independent, int G) {
+// else the streaming kernel (make_stream_plan: the least work for calls
+// flagged independent, the latency model for the others).
+Plan make_plan(const fb_weights *W, int batch, int sms, bool independent, int G, const Group &grp) {
     if (batch > 1) return make_batched_plan(W, batch, sms);
-    Plan pl = make_stream_plan(W, batch, sms, independent, G);
+    Plan pl = make_stream_plan(W, batch, sms, independent, G, grp);
     pl.tp = 1;
     pl.passes = 1;
     return pl;
 }
 
-const Plan &cached_plan(const fb_weights *W, int batch, int sms, bool independent, int G = 0) {
+const Plan &cached_plan(const fb_weights *W, int batch, int sms, bool independent, int G = 0,
+                        const Group *group = nullptr) {
     struct Entry {
         PlanKey key;
         Plan plan;
     };
     thread_local Entry memo[16];
     thread_local int used = 0, next = 0;
-    const PlanKey key{W->M, W->N, W->K, W->g, W->nS, W->nS > 0 ? W->Ks : 0, batch, sms, G, independent};
+    Group grp;
+    if (group) grp = *group;
+    else grp.M[0] = W->M;
+    PlanKey key{W->M, W->N, W->K, W->g, W->nS, W->nS > 0 ? W->Ks : 0, batch, sms, G, independent, {0, 0, 0, 0}};
+    std::copy(grp.M, grp.M + kMaxGroup, key.rows);
     for (int i = 0; i < used; ++i)
         if (memo[i].key == key) return memo[i].plan;
     Entry &e = memo[next];
     e.key = key;
-    e.plan = make_plan(W, batch, sms, independent, G);
+    e.plan = make_plan(W, batch, sms, independent, G, grp);
     next = (next + 1) % 16;
     used = std::min(used + 1, 16);
     return e.plan;
@@ -1352,10 +1390,14 @@ static fb_status launch_gemv(const fb_weights *const *Ws, int n, const void *X, 
         if (!aligned(Y[m], 4)) return FB_ERR_MISALIGNED;
         M_max = std::max(M_max, Ws[m]->M);
     }
-    // the plan of the largest matrix (the format, hence the panels, is shared)
+    // the plan of the largest matrix (the format, hence the panels, is
+    // shared), its row blocks counted over the whole group
     fb_weights Wp = *W;
     Wp.M = M_max;
-    const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0, G);
+    Group grp;
+    grp.n = n;
+    for (int m = 0; m < n; ++m) grp.M[m] = Ws[m]->M;
+    const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0, G, &grp);
     if (pl.smem > kMaxDynSmem) return FB_ERR_UNSUPPORTED;   // (no plan asks for more; a guard)
     const KernelFn fn = pl.kind == 1 ? pick_stream(t, pl.nwarps, pl.items) : pick_batched(t, pl.items);
     if (!prepare_kernel(fn, pl.smem)) return FB_ERR_CUDA;

@@ -200,8 +200,9 @@ def test_launch_plan_fits_at_the_abi_corners(L, M, N, K, nS, Ks, batch, flags):
 def test_launch_plan_shapes_by_call_kind(L):
     """Batch-1 calls get the 8-warp streaming CTA (two per SM) with rows in
     whole chunks per warp; calls flagged independent take row blocks of up to
-    32 chunks; dependent calls at most one CTA per SM.  Batched calls (8-warp
-    CTAs, eight tokens per pass) fill the SMs twice at most."""
+    32 chunks; dependent calls one wave of clusters at two CTAs per SM, in
+    clusters of 1, 2, 3, 4, 6, 8, 10, 12 or 16.  Batched calls (8-warp CTAs,
+    eight tokens per pass) fill the SMs twice at most."""
     for M, N, K, g, nS, Ks in ((4096, 4096, 2, 4, 128, 2), (11008, 4096, 2, 4, 123, 2), (8192, 8192, 3, 8, 410, 2)):
         s = fake_weights(M=M, N=N, K=K, g=g, nS=nS, Ks=Ks)
         ind = fb.fb_gemv_launch_plan(s, 1, 3, 148)
@@ -209,7 +210,7 @@ def test_launch_plan_shapes_by_call_kind(L):
         bat = fb.fb_gemv_launch_plan(s, 16, 1, 148)
         assert ind["warps"] == 8 and ind["cpb"] <= 32
         assert dep["warps"] == 8 and dep["cpb"] <= 32 and dep["cpb"] % 8 == 0
-        assert dep["C"] * dep["RB"] <= 148            # one CTA per SM: the next call takes the other half
+        assert dep["C"] * dep["RB"] <= 2 * 148 and dep["C"] in (1, 2, 3, 4, 6, 8, 10, 12, 16)
         assert bat["warps"] == 8 and bat["C"] * bat["RB"] * 2 <= 2 * 148   # 16 tokens: two passes
 
 
