@@ -271,8 +271,9 @@ FB_API fb_status fb_device_errors(unsigned int *flags, int clear);
  *   score[j] = (sum_t X[t][j]^2) * (sum_i W[i][j]^2)          j < N, fp32 out
  *   s_idx    = the nS columns of largest score (equal scores: the lower
  *              column first), in ascending order              uint32 [nS] out
- * 1 <= N <= 65536 (the selection runs in one block: O(N^2 / 1024) compares
- * per thread), 0 <= nS <= N, ldw, ldx >= N.  s_idx may be NULL when nS = 0.
+ * 1 <= N <= 2^20 (the selection runs in one block: a radix select of the
+ * score of rank nS - 1, then one ordered pass placing the selected columns),
+ * 0 <= nS <= N, ldw, ldx >= N.  s_idx may be NULL when nS = 0.
  * Returns FB_ERR_INVALID_VALUE / FB_ERR_MISALIGNED (4-byte alignment) for bad
  * arguments, FB_ERR_CUDA if a launch fails. */
 FB_API fb_status fb_fit_saliency(const float *W, int M, int N, int ldw, const float *X, int T, int ldx, int nS,

@@ -268,7 +268,8 @@ def test_fit_calls_reject_bad_arguments(L):
     sal = L.fb_fit_saliency
     assert sal(None, 8, 64, 64, F, 4, 64, 3, F, F, None) == INVALID            # no W
     assert sal(F, 0, 64, 64, F, 4, 64, 3, F, F, None) == INVALID               # M = 0
-    assert sal(F, 8, 65537, 65537, F, 4, 65537, 3, F, F, None) == INVALID      # N past the one-block selection
+    big = (1 << 20) + 1
+    assert sal(F, 8, big, big, F, 4, big, 3, F, F, None) == INVALID            # N past 2^20
     assert sal(F, 8, 64, 63, F, 4, 64, 3, F, F, None) == INVALID               # ldw < N
     assert sal(F, 8, 64, 64, F, 4, 64, 65, F, F, None) == INVALID              # nS > N
     assert sal(F, 8, 64, 64, F, 4, 64, 3, F, None, None) == INVALID            # nS > 0 without s_idx

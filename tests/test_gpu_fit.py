@@ -99,6 +99,28 @@ def test_fit_saliency_equal_scores_take_the_lower_column():
     assert s_idx.cpu().tolist() == list(range(7))
 
 
+@pytest.mark.parametrize("M,N,T,nS,levels", [(16, 5000, 2, 1234, 3), (8, 65536, 2, 4096, 7), (4, 100003, 1, 50001, 2),
+                                             (32, 4096, 4, 128, 0), (8, 777, 3, 777, 4)])
+def test_fit_saliency_selection_is_exact_on_its_scores(M, N, T, nS, levels):
+    """The selection itself, bit for bit: on the GPU's own fp32 scores, the
+    nS largest with equal scores taken lower column first (a stable sort of
+    the negated scores), ascending.  levels > 0: W in {0, 1} with `levels`
+    distinct column counts of ones, so most scores tie exactly and the cut
+    falls inside a run of equal scores."""
+    rng = np.random.default_rng(N + nS)
+    if levels:
+        ones_per_col = rng.integers(0, levels, N)
+        W = (np.arange(M)[:, None] < ones_per_col[None, :]).astype(np.float32)
+        X = np.ones((T, N), np.float32)
+    else:
+        fi = wl.fit_inputs(M, N, T=T, seed=N)
+        W, X = fi.W, fi.X
+    score, s_idx = fb.fb_fit_saliency(_gpu(W), _gpu(X), nS)
+    sc = score.cpu().numpy()
+    want = np.sort(np.argsort(-sc, kind="stable")[:nS])
+    assert np.array_equal(s_idx.cpu().numpy().astype(np.int64), want)
+
+
 def test_fit_end_to_end_4096():
     """The whole fit of a 4096 x 4096 layer (K = 2, Ks = 2, 128 salient
     columns, 8 sweeps): the same salient set, global scales within 1e-4, the
