@@ -61,6 +61,8 @@ def parse():
                     help="small case for ncu: 32 weight sets (142 MB), one pass per step, headline graph only")
     ap.add_argument("--dependent", action="store_true",
                     help="with --profile: the graph as a dependent chain (the dependent-call plan)")
+    ap.add_argument("--profile-batched", action="store_true",
+                    help="for ncu: batch-16 calls on two 8192^2 K=3 layers (a few calls, independent flags)")
     ap.add_argument("--profile-fit", action="store_true",
                     help="for ncu --profile-from-start off: one whole 4096^2 fit inside a profiler range, nothing else")
     return ap.parse_args()
@@ -334,6 +336,9 @@ def run_ours(args):
 
     if args.profile_fit:
         profile_fit(device)
+        return
+    if args.profile_batched:
+        profile_batched(device)
         return
 
     global WEIGHT_SETS, PASSES_PER_STEP
@@ -656,6 +661,25 @@ def bench_group_scales(args, device, stream, world, peak):
         gbs = nbytes / (us * 1e-6) / 1e9
         out[name] = {"gemv_us": round(us, 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
     return out
+
+
+def profile_batched(device):
+    """A small case of the batched kernel for ncu: batch-16 calls on two
+    8192 x 8192 K = 3 layers (5% salient columns), three passes over both,
+    eagerly (PDL + FB_GEMV_INDEPENDENT)."""
+    import torch
+    import lut_binary_gemv_b200 as fb
+    import workloads as wl
+    ps = [wl.layer70b(0, 16)] + [wl.make_problem(8192, 8192, 3, g=8, nS=wl.salient_count(0.05, 8192), Ks=2,
+                                                 batch=16, x_dtype="f16", alpha_dist="small", seed=(7, 0, 1))]
+    Ws = [fb.Weights.from_problem(p, device=device) for p in ps]
+    Xs = [torch.from_numpy(p.x).to(device) for p in ps]
+    Ys = [torch.empty((16, p.M), dtype=torch.float32, device=device) for p in ps]
+    for _ in range(3):
+        for W, X, Y in zip(Ws, Xs, Ys):
+            fb.fb_gemv_batched(W, X, Y=Y, flags=fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_batched": True, "calls": 6}), flush=True)
 
 
 FIT_SHAPE = dict(M=4096, N=4096, K=2, Ks=2, nS=128, sweeps=8, T=64)

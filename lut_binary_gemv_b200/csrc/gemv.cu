@@ -637,31 +637,38 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
     }
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-    // ---- 1. before the wait: panel 0's words and row scales, the column
-    // sources of panel 0 (and its x when independent) ----------------------
-    // One register set: right after an item's lookups, its registers take
-    // the same item of the next panel, so each load has a panel's time to
-    // land (two alternating sets would give no more lead).
-    uint32_t w[I][8];
-    float rar[I];
-    auto load_item = [&](int i, const PanelDesc &d) {
+    // ---- 1. before the wait: the first D panels' words and row scales, the
+    // column sources of panel 0 (and its x when independent) ---------------
+    // A ring of D register sets (D * I = 4 items for I <= 4): right after an
+    // item's lookups in panel v, its registers take the same item of panel v
+    // + D, so each load has D panels' time to land; a CTA with at most D
+    // panels has all its words requested before the wait.
+    constexpr int D = I == 1 ? 4 : I == 2 ? 2 : 1;
+    uint32_t w[D][I][8];
+    float rar[D][I];
+    auto load_item = [&](auto slotc, int i, const PanelDesc &d) {
+        constexpr int sl = decltype(slotc)::value;
         const int Bp = desc_bp(d);
         const size_t blk = 32u * (unsigned)Bp;
         const int cl = warp + NW * i;
         const int row = (c_first + cl) * kChunkRows + lane;
-        rar[i] = cl < nvalid && row < a.M ? __ldg(row_scales(a, d.kb) + row) : 0.0f;
+        rar[sl][i] = cl < nvalid && row < a.M ? __ldg(row_scales(a, d.kb) + row) : 0.0f;
         if (cl < nvalid) {
             const uint8_t *p = d.pl + blk * (size_t)(c_first + cl);
             if (Bp == 32) {
                 const uint4 x0 = ldg_stream(p + 16 * lane), x1 = ldg_stream(p + 512 + 16 * lane);
-                w[i][0] = x0.x; w[i][1] = x0.y; w[i][2] = x0.z; w[i][3] = x0.w;
-                w[i][4] = x1.x; w[i][5] = x1.y; w[i][6] = x1.z; w[i][7] = x1.w;
+                w[sl][i][0] = x0.x; w[sl][i][1] = x0.y; w[sl][i][2] = x0.z; w[sl][i][3] = x0.w;
+                w[sl][i][4] = x1.x; w[sl][i][5] = x1.y; w[sl][i][6] = x1.z; w[sl][i][7] = x1.w;
             } else {
                 const Words r = load_item_narrow(p, Bp, lane);
 #pragma unroll
-                for (int m = 0; m < 8; ++m) w[i][m] = r.w[m];
+                for (int m = 0; m < 8; ++m) w[sl][i][m] = r.w[m];
             }
         }
+    };
+    auto load_panel = [&](auto slotc, const PanelDesc &d) {
+#pragma unroll
+        for (int i = 0; i < I; ++i) load_item(slotc, i, d);
     };
     if (tid < kDescRing - 4 && tid < n_v) s_ring[tid] = panel_desc(a, vb + tid);
     Staged st[2] = {{0.0f, 0u, -1}, {0.0f, 0u, -1}};
@@ -673,15 +680,17 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
     PanelDesc d1;
     if (n_v > 0) {
         const PanelDesc d0 = panel_desc(a, vb);
-#pragma unroll
-        for (int i = 0; i < I; ++i) load_item(i, d0);
+        load_panel(std::integral_constant<int, 0>{}, d0);
         stage(st[0], d0, independent);
     }
     if (n_v > 1) d1 = panel_desc(a, vb + 1);
+    if (D > 1 && n_v > 1) load_panel(std::integral_constant<int, (D > 1 ? 1 : 0)>{}, d1);
+    if (D > 2 && n_v > 2) load_panel(std::integral_constant<int, (D > 2 ? 2 : 0)>{}, panel_desc(a, vb + 2));
+    if (D > 3 && n_v > 3) load_panel(std::integral_constant<int, (D > 3 ? 3 : 0)>{}, panel_desc(a, vb + 3));
     if (!independent) {
         // the rest of the slice into L2 while the previous kernel finishes
         if (tid == 0) {
-            for (int v = 1; v < min(n_v, 8); ++v) {
+            for (int v = D; v < min(n_v, 8); ++v) {
                 const PanelDesc d = panel_desc(a, vb + v);
                 const uint32_t blk = 32u * (uint32_t)desc_bp(d);
                 prefetch_l2(d.pl + (size_t)blk * c_first, blk * (uint32_t)nvalid);
@@ -705,8 +714,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
     for (int i = 0; i < I; ++i) racc[i] = 0.0f;
 
     // ---- 2. per panel: tables, then this warp's items ----------------------
-    auto panel = [&](auto bufc, int vi) {
+    // (table buffer buf = vi % 2, register set slotc = vi % D)
+    auto panel = [&](auto bufc, auto slotc, int vi) {
         constexpr int buf = decltype(bufc)::value;
+        constexpr int sl = decltype(slotc)::value;
         const int Bp = desc_bp(s_ring[vi % kDescRing]);
         float *tb = tables + 32 * buf;
         build_byte_table<NW>(zbuf + buf * kPanelCols, tb, warp, lane);
@@ -715,23 +726,23 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
         if (vi + 2 < n_v) resolve(st[buf]);   // panel vi + 2, staged one panel ago
         if (tid == 0 && vi + 4 < n_v) s_ring[(vi + 4) % kDescRing] = panel_desc(a, vb + vi + 4);
         __syncthreads();   // tables of panel vi complete; every warp done with panel vi - 1
-        const bool more = vi + 1 < n_v;
-        const PanelDesc &nd = s_ring[(vi + 1) % kDescRing];   // the next panel (its items load here)
+        const bool more = vi + D < n_v;
+        const PanelDesc &nd = s_ring[(vi + D) % kDescRing];   // panel vi + D (its items load here)
         if (Bp == 32) {
 #pragma unroll
             for (int i = 0; i < I; i += 2) {
                 const int c0 = warp + NW * i;
                 if (i + 1 < I && c0 + NW < nvalid) {
                     float s0, s1;
-                    lookup_rows2(w[i], w[i + 1], off_full, tb, s0, s1);
-                    racc[i] = __fadd_rn(racc[i], __fmul_rn(rar[i], s0));
-                    racc[i + 1] = __fadd_rn(racc[i + 1], __fmul_rn(rar[i + 1], s1));
+                    lookup_rows2(w[sl][i], w[sl][i + 1], off_full, tb, s0, s1);
+                    racc[i] = __fadd_rn(racc[i], __fmul_rn(rar[sl][i], s0));
+                    racc[i + 1] = __fadd_rn(racc[i + 1], __fmul_rn(rar[sl][i + 1], s1));
                 } else if (c0 < nvalid) {
-                    racc[i] = __fadd_rn(racc[i], __fmul_rn(rar[i], lookup_row(w[i], off_full, tb)));
+                    racc[i] = __fadd_rn(racc[i], __fmul_rn(rar[sl][i], lookup_row(w[sl][i], off_full, tb)));
                 }
                 if (more) {
-                    load_item(i, nd);
-                    if (i + 1 < I) load_item(i + 1, nd);
+                    load_item(slotc, i, nd);
+                    if (i + 1 < I) load_item(slotc, i + 1, nd);
                 }
             }
         } else {
@@ -739,15 +750,31 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
 #pragma unroll
             for (int i = 0; i < I; ++i) {
                 if (warp + NW * i < nvalid)
-                    racc[i] = __fadd_rn(racc[i], __fmul_rn(rar[i], lookup_row_narrow(w[i], o.w, tb, Bp >> 2)));
-                if (more) load_item(i, nd);
+                    racc[i] = __fadd_rn(racc[i],
+                                        __fmul_rn(rar[sl][i], lookup_row_narrow(w[sl][i], o.w, tb, Bp >> 2)));
+                if (more) load_item(slotc, i, nd);
             }
         }
     };
+    using C0 = std::integral_constant<int, 0>;
+    using C1 = std::integral_constant<int, 1>;
+    using S1 = std::integral_constant<int, (D > 1 ? 1 : 0)>;
+    using S2 = std::integral_constant<int, (D > 2 ? 2 : 0)>;
+    using S3 = std::integral_constant<int, (D > 3 ? 3 : 0)>;
+    if constexpr (D == 4) {
 #pragma unroll 1
-    for (int vi = 0; vi < n_v; vi += 2) {
-        panel(std::integral_constant<int, 0>{}, vi);
-        if (vi + 1 < n_v) panel(std::integral_constant<int, 1>{}, vi + 1);
+        for (int vi = 0; vi < n_v; vi += 4) {   // panels vi .. vi + 3: buffers 0 1 0 1, register sets 0 1 2 3
+            panel(C0{}, C0{}, vi);
+            if (vi + 1 < n_v) panel(C1{}, S1{}, vi + 1);
+            if (vi + 2 < n_v) panel(C0{}, S2{}, vi + 2);
+            if (vi + 3 < n_v) panel(C1{}, S3{}, vi + 3);
+        }
+    } else {
+#pragma unroll 1
+        for (int vi = 0; vi < n_v; vi += 2) {   // panels vi, vi + 1: buffers 0 1, register sets vi % D
+            panel(C0{}, C0{}, vi);
+            if (vi + 1 < n_v) panel(C1{}, S1{}, vi + 1);
+        }
     }
 
     // ---- 3. the cluster's row partials, summed by their owner in rank order
@@ -1177,12 +1204,25 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         split_weighted(groups, pl.C, pl.cpb, pl.vsplit);
     };
     if (independent) {
-        // row blocks of up to 32 chunks, C = 2 for matrices of at most 8 row
-        // blocks, else 1.  (64-chunk blocks run faster on one large matrix
-        // but make each CTA live so long that graphs of mixed calls, the 7B
-        // step, lose more to filling and draining than they gain.)
-        const int RB = ceil_div(pl.nchunks, max_cpb);
-        set(RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
+        // Matrices of at least 64 MiB of packed planes (65536 items): row
+        // blocks of 64 chunks (eight per warp) in clusters of 2 -- the
+        // fewest table builds per row.  Smaller ones: row blocks of up to 32
+        // chunks, C = 2 for matrices of at most 8 row blocks, else 1 (on
+        // those, 64-chunk blocks make each CTA live so long that graphs of
+        // such calls lose more to filling and draining than they gain).
+        // Measured on B200 in graphs of independent calls: 28672x8192 and
+        // 8192x28672 with K = 3 run 12-13% faster with 64-chunk blocks,
+        // 8192^2 K = 3 9% slower, 4096^2 (the 7B-shaped matrices) slower
+        // too; C = 4 on 4096^2 loses 4% in long graphs.
+        long items = 0;
+        for (int g : groups) items += g;
+        items = items / 32 * pl.nchunks;
+        if (items >= 65536 && pl.nchunks >= 2 * max_cpb) {
+            set(2, 2 * max_cpb);
+        } else {
+            const int RB = ceil_div(pl.nchunks, max_cpb);
+            set(RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
+        }
     } else {
         // Latency model of a call that waits for its predecessor (fitted to
         // dependent chains of this kernel on B200 over the shapes 4096^2,

@@ -170,7 +170,7 @@ def test_launch_plan_covers_the_matrix(L, shape, batch, flags):
     assert plan["V"] == V
     assert 1 <= plan["C"] <= min(16, V)
     assert plan["RB"] * plan["cpb"] >= nchunks > (plan["RB"] - 1) * plan["cpb"]
-    assert plan["cpb"] <= 32
+    assert plan["cpb"] <= (64 if batch == 1 and flags == 3 else 32)   # 64: large independent calls
     assert plan["warps"] == 8
     assert 0 < plan["smem"] <= 225 * 1024
     if batch > 1:                       # the row partials of a pass fit in the 64 KB table bytes
@@ -200,7 +200,7 @@ def test_launch_plan_fits_at_the_abi_corners(L, M, N, K, nS, Ks, batch, flags):
 def test_launch_plan_shapes_by_call_kind(L):
     """Batch-1 calls get the 8-warp streaming CTA (two per SM) with rows in
     whole chunks per warp; calls flagged independent take row blocks of up to
-    32 chunks; dependent calls one wave of clusters at two CTAs per SM, in
+    32 chunks (64 from 64 MiB of packed planes); dependent calls one wave of clusters at two CTAs per SM, in
     clusters of 1, 2, 3, 4, 6, 8, 10, 12 or 16.  Batched calls (8-warp CTAs,
     eight tokens per pass) fill the SMs twice at most."""
     for M, N, K, g, nS, Ks in ((4096, 4096, 2, 4, 128, 2), (11008, 4096, 2, 4, 123, 2), (8192, 8192, 3, 8, 410, 2)):
@@ -208,7 +208,7 @@ def test_launch_plan_shapes_by_call_kind(L):
         ind = fb.fb_gemv_launch_plan(s, 1, 3, 148)
         dep = fb.fb_gemv_launch_plan(s, 1, 1, 148)
         bat = fb.fb_gemv_launch_plan(s, 16, 1, 148)
-        assert ind["warps"] == 8 and ind["cpb"] <= 32
+        assert ind["warps"] == 8 and ind["cpb"] <= (64 if M * N * K >= 64 * 8 * 2**20 else 32)
         assert dep["warps"] == 8 and dep["cpb"] <= 32 and dep["cpb"] % 8 == 0
         assert dep["C"] * dep["RB"] <= 2 * 148 and dep["C"] in (1, 2, 3, 4, 6, 8, 10, 12, 16)
         assert bat["warps"] == 8 and bat["C"] * bat["RB"] * 2 <= 2 * 148   # 16 tokens: two passes
