@@ -639,11 +639,14 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
 
     // ---- 1. before the wait: the first D panels' words and row scales, the
     // column sources of panel 0 (and its x when independent) ---------------
-    // A ring of D register sets (D * I = 4 items for I <= 4): right after an
-    // item's lookups in panel v, its registers take the same item of panel v
-    // + D, so each load has D panels' time to land; a CTA with at most D
-    // panels has all its words requested before the wait.
-    constexpr int D = I == 1 ? 4 : I == 2 ? 2 : 1;
+    // A ring of D register sets (two for warps of one or two items, whose
+    // panels are short; one for more): right after an item's lookups in panel
+    // v, its registers take the same item of panel v + D, so each load has D
+    // panels' time to land, and a CTA of one or two panels has all its words
+    // requested before the wait.  (Four sets for one item lengthened the
+    // dependent chain of a 7B-shaped layer, whose calls alternate between
+    // kernels, by 7%: the four-panel loop body is twice the code.)
+    constexpr int D = I <= 2 ? 2 : 1;
     uint32_t w[D][I][8];
     float rar[D][I];
     auto load_item = [&](auto slotc, int i, const PanelDesc &d) {
@@ -684,9 +687,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
         stage(st[0], d0, independent);
     }
     if (n_v > 1) d1 = panel_desc(a, vb + 1);
-    if (D > 1 && n_v > 1) load_panel(std::integral_constant<int, (D > 1 ? 1 : 0)>{}, d1);
-    if (D > 2 && n_v > 2) load_panel(std::integral_constant<int, (D > 2 ? 2 : 0)>{}, panel_desc(a, vb + 2));
-    if (D > 3 && n_v > 3) load_panel(std::integral_constant<int, (D > 3 ? 3 : 0)>{}, panel_desc(a, vb + 3));
+    if (D > 1 && n_v > 1) load_panel(std::integral_constant<int, D - 1>{}, d1);
     if (!independent) {
         // the rest of the slice into L2 while the previous kernel finishes
         if (tid == 0) {
@@ -758,23 +759,11 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
     };
     using C0 = std::integral_constant<int, 0>;
     using C1 = std::integral_constant<int, 1>;
-    using S1 = std::integral_constant<int, (D > 1 ? 1 : 0)>;
-    using S2 = std::integral_constant<int, (D > 2 ? 2 : 0)>;
-    using S3 = std::integral_constant<int, (D > 3 ? 3 : 0)>;
-    if constexpr (D == 4) {
+    using S1 = std::integral_constant<int, D - 1>;
 #pragma unroll 1
-        for (int vi = 0; vi < n_v; vi += 4) {   // panels vi .. vi + 3: buffers 0 1 0 1, register sets 0 1 2 3
-            panel(C0{}, C0{}, vi);
-            if (vi + 1 < n_v) panel(C1{}, S1{}, vi + 1);
-            if (vi + 2 < n_v) panel(C0{}, S2{}, vi + 2);
-            if (vi + 3 < n_v) panel(C1{}, S3{}, vi + 3);
-        }
-    } else {
-#pragma unroll 1
-        for (int vi = 0; vi < n_v; vi += 2) {   // panels vi, vi + 1: buffers 0 1, register sets vi % D
-            panel(C0{}, C0{}, vi);
-            if (vi + 1 < n_v) panel(C1{}, S1{}, vi + 1);
-        }
+    for (int vi = 0; vi < n_v; vi += 2) {   // panels vi, vi + 1: buffers 0 1, register sets vi % D
+        panel(C0{}, C0{}, vi);
+        if (vi + 1 < n_v) panel(C1{}, S1{}, vi + 1);
     }
 
     // ---- 3. the cluster's row partials, summed by their owner in rank order
