@@ -479,8 +479,15 @@ __device__ __forceinline__ void lookup_rows2(const uint32_t (&wa)[8], const uint
     sb = __fadd_rn(__fadd_rn(f2sum(acc_b[0]), f2sum(acc_b[1])), __fadd_rn(f2sum(acc_b[2]), f2sum(acc_b[3])));
 }
 
+// Where column t of a panel keeps its z in the z buffer: the low four
+// columns of every 8-column group first (group q at 4q), then the high four
+// (at 128 + 4q), so that lane q reads its group as two 16-byte words at
+// consecutive addresses across the warp (4 wavefronts each, not 8).
+__device__ __forceinline__ int z_slot(int t) { return ((t & 4) ? kPanelCols / 2 : 0) + 4 * (t >> 3) + (t & 3); }
+
 // LUT-BSF for one virtual panel, built by the whole CTA: lane q builds byte
-// group q (columns 8q .. 8q+7, z in zp), warp w its entries b = 32w .. 32w+31:
+// group q (columns 8q .. 8q+7, their z at z_slot in zp), warp w its entries
+// b = 32w .. 32w+31:
 // entry b = T_lo[b & 15] + T_hi[b >> 4], where T_lo and T_hi are the 16-entry
 // tables of the group's low and high 4 columns, each (+-z0 +- z1) + (+-z2 +-
 // z3).  Columns past a narrow panel's width have z = 0, so their entries are
@@ -489,8 +496,8 @@ __device__ __forceinline__ void lookup_rows2(const uint32_t (&wa)[8], const uint
 template <int NW>
 __device__ __forceinline__ void build_byte_table(const float *zp, float *T, int warp, int lane) {
     constexpr int kHi = 16 / NW;   // high-nibble values per warp: entries b = 16*kHi*warp ...
-    const float4 za = *reinterpret_cast<const float4 *>(zp + 8 * lane);
-    const float4 zb = *reinterpret_cast<const float4 *>(zp + 8 * lane + 4);
+    const float4 za = *reinterpret_cast<const float4 *>(zp + 4 * lane);
+    const float4 zb = *reinterpret_cast<const float4 *>(zp + kPanelCols / 2 + 4 * lane);
     float lo[16];
     sums16(za.x, za.y, za.z, za.w, lo);
     float hi[kHi];
@@ -703,7 +710,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
     if (n_v > 1) stage(st[1], d1, true);   // x of panel 1 in flight with panel 0's
     resolve(st[0]);
     if (n_v > 1) resolve(st[1]);
-    if (kAllStage || tid < kPanelCols) zbuf[tid] = z_of(st[0]);
+    if (kAllStage || tid < kPanelCols) zbuf[z_slot(tid)] = z_of(st[0]);
     __syncthreads();   // z of panel 0 and the first descriptors written
     if (n_v > 2) stage(st[0], s_ring[2], true);
 
@@ -722,7 +729,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_c
         const int Bp = desc_bp(s_ring[vi % kDescRing]);
         float *tb = tables + 32 * buf;
         build_byte_table<NW>(zbuf + buf * kPanelCols, tb, warp, lane);
-        if (vi + 1 < n_v && (kAllStage || tid < kPanelCols)) zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
+        if (vi + 1 < n_v && (kAllStage || tid < kPanelCols))
+            zbuf[(buf ^ 1) * kPanelCols + z_slot(tid)] = z_of(st[buf ^ 1]);
         if (vi + 3 < n_v) stage(st[buf ^ 1], s_ring[(vi + 3) % kDescRing], true);
         if (vi + 2 < n_v) resolve(st[buf]);   // panel vi + 2, staged one panel ago
         if (tid == 0 && vi + 4 < n_v) s_ring[(vi + 4) % kDescRing] = panel_desc(a, vb + vi + 4);
@@ -902,7 +910,7 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
     if (S > 1) stage(1, d0, 1, true);   // step 1: panel 0 (a pass holds at least two tokens)
     resolve(0);
     if (S > 1) resolve(1);
-    zbuf[tid] = z_of(st[0]);
+    zbuf[z_slot(tid)] = z_of(st[0]);
     __syncthreads();   // z of step 0, the first descriptors and the zeroed partials written
     if (S > 2) stage(0, TP > 2 ? d0 : d1, 2 % TP, true);
 
@@ -917,7 +925,7 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
         const int Bp = desc_bp(s_ring[vi % kDescRing]);
         float *tb = tables + 32 * buf;
         if (tok < nt) build_byte_table<NW>(zbuf + buf * kPanelCols, tb, warp, lane);
-        if (s2 + 1 < S) zbuf[(buf ^ 1) * kPanelCols + tid] = z_of(st[buf ^ 1]);
+        if (s2 + 1 < S) zbuf[(buf ^ 1) * kPanelCols + z_slot(tid)] = z_of(st[buf ^ 1]);
         if (s2 + 3 < S) {
             const int s3 = s2 + 3, v3 = s3 / TP;
             stage(buf ^ 1, s_ring[v3 % kDescRing], s3 - v3 * TP, true);
