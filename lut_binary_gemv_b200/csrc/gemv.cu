@@ -12,19 +12,20 @@
 // panels (balanced by their lookup work), so the cluster covers every column
 // of its rows.
 //
-// stream_kernel (batch 1; 8 warps, two CTAs per SM, or 16 warps, one):
-//   1. the words of the CTA's first two panels are loaded straight into
-//      registers (each lane its rows' bytes, 128-bit loads), with the row
-//      scales; for calls that depend on the previous kernel this, and an L2
-//      prefetch of the rest of the slice, happens before the
-//      programmatic-launch wait, and x is read after it;
+// stream_kernel (batch 1; 8 warps, three CTAs per SM for calls flagged
+// independent and two otherwise, or 16 warps, one):
+//   1. the words of the CTA's first panel (two for warps of one or two
+//      items) are loaded straight into registers (each lane its rows' bytes,
+//      128-bit loads), with the row scales; for calls that depend on the
+//      previous kernel this, and an L2 prefetch of the next panels, happens
+//      before the programmatic-launch wait, and x is read after it;
 //   2. per panel, the CTA builds the panel's byte tables in shared memory
 //      (LUT-BSF: z = alpha_c * x, salient panels reading x[s_idx[t]] -- the
 //      virtual columnar mapping -- and for each group of 8 columns the 256
 //      sums sum_t (bit t of b ? +z_t : -z_t), each the sum of the two 4-column
 //      tables of its nibbles), double-buffered, one CTA barrier per panel;
-//      meanwhile the words of the panel after next load into the register
-//      set the previous panel used;
+//      right after an item's lookups its registers take the same item of a
+//      later panel;
 //   3. each lane walks its row's bytes: one `prmt` merges a weight byte and
 //      the lane's column offset into a table address, one shared load fetches
 //      the partial sum, packed fp32x2 adds accumulate (a gather-add, no tensor
@@ -577,9 +578,15 @@ __device__ __noinline__ Words load_item_narrow(const uint8_t *blk, int Bp, int l
 constexpr int kStreamWarps = 8;
 constexpr int kDescRing = 8;   // panel descriptors kept in shared memory (a ring)
 
-template <int XT, int NW, int I>
-__global__ void __launch_bounds__(NW * 32, 16 / NW) stream_kernel(const __grid_constant__ GemvArgs args) {
-    static_assert(NW == 8 || NW == 16, "8 warps (two CTAs per SM) or 16 (one)");
+// CTAs per SM the kernel is compiled for (its register budget): three for
+// calls flagged independent with up to four items per warp (80 registers,
+// 24 warps per SM: the overlapped calls' latency is hidden by more warps),
+// two otherwise (128 registers: a call that waits for its predecessor is
+// bound by each CTA's own critical path, and keeps an SM slot free for the
+// next call's CTAs).
+template <int XT, int NW, int I, int kBlocks>
+__global__ void __launch_bounds__(NW * 32, kBlocks) stream_kernel(const __grid_constant__ GemvArgs args) {
+    static_assert(NW == 8 || NW == 16, "8 warps (two or three CTAs per SM) or 16 (one)");
     constexpr bool kAllStage = NW * 32 == kPanelCols;   // every thread stages a column
     extern __shared__ __align__(128) float smem_f[];
     __shared__ __align__(16) GemvArgs s_args;
@@ -1015,14 +1022,19 @@ KernelFn pick_batched(fb_dtype t, int items) {
                       : items == 4 ? pick_batched_xt<4>(t) : pick_batched_xt<8>(t);
 }
 
-template <int NW, int I>
+template <int NW, int I, int B = 16 / NW>
 KernelFn pick_stream_xt(fb_dtype t) {
-    return t == FB_F32 ? stream_kernel<FB_F32, NW, I> : t == FB_F16 ? stream_kernel<FB_F16, NW, I>
-                                                                    : stream_kernel<FB_BF16, NW, I>;
+    return t == FB_F32 ? stream_kernel<FB_F32, NW, I, B> : t == FB_F16 ? stream_kernel<FB_F16, NW, I, B>
+                                                                       : stream_kernel<FB_BF16, NW, I, B>;
 }
-KernelFn pick_stream(fb_dtype t, int nw, int items) {
+// The streaming kernel for nw warps and `items` chunks per warp; `three`:
+// the variant with three CTAs per SM (independent calls, up to four items).
+KernelFn pick_stream(fb_dtype t, int nw, int items, bool three) {
     if (nw == 16) return items == 1 ? pick_stream_xt<16, 1>(t) : items == 2 ? pick_stream_xt<16, 2>(t)
                                                                              : pick_stream_xt<16, 4>(t);
+    if (three && items <= 4)
+        return items == 1 ? pick_stream_xt<8, 1, 3>(t) : items == 2 ? pick_stream_xt<8, 2, 3>(t)
+                                                                    : pick_stream_xt<8, 4, 3>(t);
     return items == 1 ? pick_stream_xt<8, 1>(t) : items == 2 ? pick_stream_xt<8, 2>(t)
                       : items == 4 ? pick_stream_xt<8, 4>(t) : pick_stream_xt<8, 8>(t);
 }
@@ -1172,8 +1184,9 @@ size_t stream_smem(int cpb) {
 
 int stream_items(int cpb, int nw = kStreamWarps) { return cpb <= nw ? 1 : cpb <= 2 * nw ? 2 : cpb <= 4 * nw ? 4 : 8; }
 
-// Plan of the streaming kernel (8 warps, two CTAs per SM, up to 4 chunks per
-// warp -- 8 with the tuning override -- and clusters of up to 16 CTAs).
+// Plan of the streaming kernel (8 warps, up to 4 chunks per warp -- 8 for
+// the largest independent calls and with the tuning override -- and
+// clusters of up to 16 CTAs).
 //  * Independent calls overlap their neighbours: row blocks of 32 chunks
 //    (few table builds per row), C = 2 for matrices of at most 8 row
 //    blocks, else 1.
@@ -1377,6 +1390,12 @@ bool prepare_kernel(KernelFn fn, size_t smem) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want) != cudaSuccess)
         return false;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) return false;
+    // all of the unified L1 / shared-memory array as shared memory, so that
+    // three CTAs of ~72 KB fit on an SM (the kernels' own global loads bypass
+    // or barely use L1)
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+        cudaSuccess)
+        return false;
     if (n_done < 64) done[n_done++] = {fn, dev, want};
     return true;
 }
@@ -1436,7 +1455,8 @@ static fb_status launch_gemv(const fb_weights *const *Ws, int n, const void *X, 
     for (int m = 0; m < n; ++m) grp.M[m] = Ws[m]->M;
     const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0, G, &grp);
     if (pl.smem > kMaxDynSmem) return FB_ERR_UNSUPPORTED;   // (no plan asks for more; a guard)
-    const KernelFn fn = pl.kind == 1 ? pick_stream(t, pl.nwarps, pl.items) : pick_batched(t, pl.items);
+    const KernelFn fn = pl.kind == 1 ? pick_stream(t, pl.nwarps, pl.items, (flags & FB_GEMV_INDEPENDENT) != 0)
+                                     : pick_batched(t, pl.items);
     if (!prepare_kernel(fn, pl.smem)) return FB_ERR_CUDA;
 
     GemvArgs a;
