@@ -826,12 +826,13 @@ __global__ void __launch_bounds__(NW * 32, kBlocks) stream_kernel(const __grid_c
 // Shared memory: tables (two interleaved buffers, 64 KB; after the last
 // lookups the same bytes receive the cluster's row partials) | z of two
 // steps | row partials [tp][R].  8 warps; with 8 tokens per pass two CTAs
-// share an SM.
+// share an SM (128 registers); with 2 tokens per pass, three (kBlocks = 3:
+// 80 registers, up to four items per warp).
 constexpr int kBatchWarps = 8;
 constexpr int kMaxTokensPerPass = 16;
 
-template <int XT, int I>
-__global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __grid_constant__ GemvArgs args) {
+template <int XT, int I, int kBlocks>
+__global__ void __launch_bounds__(kBatchWarps * 32, kBlocks) batched_kernel(const __grid_constant__ GemvArgs args) {
     constexpr int NW = kBatchWarps, NT = NW * 32;
     extern __shared__ __align__(128) float smem_f[];
     __shared__ __align__(16) GemvArgs s_args;
@@ -1013,11 +1014,17 @@ __global__ void __launch_bounds__(kBatchWarps * 32, 2) batched_kernel(const __gr
 
 using KernelFn = void (*)(GemvArgs);
 
-template <int I>
+template <int I, int B = 2>
 KernelFn pick_batched_xt(fb_dtype t) {
-    return t == FB_F32 ? batched_kernel<FB_F32, I> : t == FB_F16 ? batched_kernel<FB_F16, I> : batched_kernel<FB_BF16, I>;
+    return t == FB_F32 ? batched_kernel<FB_F32, I, B> : t == FB_F16 ? batched_kernel<FB_F16, I, B>
+                                                                    : batched_kernel<FB_BF16, I, B>;
 }
-KernelFn pick_batched(fb_dtype t, int items) {
+// The batched kernel for `items` chunks per warp; `three`: the variant with
+// three CTAs per SM (up to four items).
+KernelFn pick_batched(fb_dtype t, int items, bool three) {
+    if (three && items <= 4)
+        return items == 1 ? pick_batched_xt<1, 3>(t) : items == 2 ? pick_batched_xt<2, 3>(t)
+                                                                   : pick_batched_xt<4, 3>(t);
     return items == 1 ? pick_batched_xt<1>(t) : items == 2 ? pick_batched_xt<2>(t)
                       : items == 4 ? pick_batched_xt<4>(t) : pick_batched_xt<8>(t);
 }
@@ -1061,6 +1068,7 @@ struct Plan {
     int kind;    // 1: stream_kernel; 2: batched_kernel
     int items;   // stream / batched kernel: chunks per warp per panel
     int tp, passes;   // batched kernel: tokens per pass, passes (grid.z)
+    int three = 0;    // batched kernel: the variant with three CTAs per SM
     int vsplit[kMaxCluster + 1];
     size_t smem;
 };
@@ -1288,9 +1296,10 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
 }
 
 // Plan of the batched kernel (8 warps): row blocks of up to 32 chunks, an
-// even number of tokens per pass (8 by default: two CTAs share an SM; 16
-// with FB_PLAN's third field), and as many CTAs per cluster (up to 16) as
-// fill the SMs twice.
+// even number of tokens per pass (2 for matrices of at most 32 MiB of packed
+// planes, three CTAs per SM; else up to 8, two CTAs per SM; up to 16 with
+// FB_PLAN's third field), and as many CTAs per cluster (up to 16) as fill
+// the SMs' CTA slots once.
 size_t batched_smem(int cpb, int tp) {
     return (size_t)kTableBytes + kZBytes + (size_t)tp * cpb * kChunkRows * 4;
 }
@@ -1308,7 +1317,19 @@ Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
     pl.kind = 2;
     int tp_max = 8, oc = 0, ocpb = 0, otp = 0;
     const char *ov = getenv("FB_PLAN");
-    if (ov && sscanf(ov, "%d,%d,%d", &oc, &ocpb, &otp) >= 2 && otp >= 2) tp_max = std::min(otp, kMaxTokensPerPass);
+    const bool tuned = ov && sscanf(ov, "%d,%d,%d", &oc, &ocpb, &otp) >= 2;
+    if (tuned && otp >= 2) tp_max = std::min(otp, kMaxTokensPerPass);
+    // Matrices of at most 32 MiB of packed planes stay in L2 while the passes
+    // stream them together, so they take passes of 2 tokens in the variant
+    // with three CTAs per SM (24 warps; a pass's partials and tables fit in
+    // 74 KB): more passes, but their weight reads hit L2 and the extra warps
+    // hide the per-token barrier latency (8192^2 K=3 at batch 16 on B200:
+    // 146.7 -> 111.9 us).  Larger ones keep passes of up to 8 tokens (two
+    // CTAs per SM): for 28672x8192 passes of 2 were 4-6% slower.
+    long plane_bytes = 0;
+    for (int g : groups) plane_bytes += (long)g * 32 * pl.nchunks;
+    pl.three = !tuned && plane_bytes <= (32L << 20) ? 1 : 0;
+    if (pl.three) tp_max = 2;
     tp_max &= ~1;
     pl.tp = std::min(round_up(batch, 2), tp_max);
     pl.passes = ceil_div(batch, pl.tp);
@@ -1316,7 +1337,8 @@ Plan make_batched_plan(const fb_weights *W, int batch, int sms) {
     pl.RB = ceil_div(pl.nchunks, max_cpb);
     pl.cpb = ceil_div(pl.nchunks, pl.RB);
     const long blocks = (long)pl.RB * pl.passes;
-    int C = blocks >= 2L * sms ? 1 : (int)(2L * sms / blocks);
+    const long slots = (pl.three ? 3L : 2L) * sms;   // fill the SMs' CTA slots once
+    int C = blocks >= slots ? 1 : (int)(slots / blocks);
     C = std::max(1, std::min(std::min(C, kMaxCluster), pl.V));
     if (ov && oc >= 1 && ocpb >= 1) {
         C = std::min(std::min(oc, kMaxCluster), pl.V);
@@ -1456,7 +1478,7 @@ static fb_status launch_gemv(const fb_weights *const *Ws, int n, const void *X, 
     const Plan &pl = cached_plan(&Wp, batch, sm_count(), (flags & FB_GEMV_INDEPENDENT) != 0, G, &grp);
     if (pl.smem > kMaxDynSmem) return FB_ERR_UNSUPPORTED;   // (no plan asks for more; a guard)
     const KernelFn fn = pl.kind == 1 ? pick_stream(t, pl.nwarps, pl.items, (flags & FB_GEMV_INDEPENDENT) != 0)
-                                     : pick_batched(t, pl.items);
+                                     : pick_batched(t, pl.items, pl.three != 0);
     if (!prepare_kernel(fn, pl.smem)) return FB_ERR_CUDA;
 
     GemvArgs a;

@@ -198,11 +198,12 @@ def test_launch_plan_fits_at_the_abi_corners(L, M, N, K, nS, Ks, batch, flags):
 
 
 def test_launch_plan_shapes_by_call_kind(L):
-    """Batch-1 calls get the 8-warp streaming CTA (two per SM) with rows in
-    whole chunks per warp; calls flagged independent take row blocks of up to
-    32 chunks (64 from 64 MiB of packed planes); dependent calls one wave of clusters at two CTAs per SM, in
-    clusters of 1, 2, 3, 4, 6, 8, 10, 12 or 16.  Batched calls (8-warp CTAs,
-    eight tokens per pass) fill the SMs twice at most."""
+    """Batch-1 calls get the 8-warp streaming CTA with rows in whole chunks
+    per warp; calls flagged independent take row blocks of up to 32 chunks
+    (64 from 64 MiB of packed planes); dependent calls one wave of clusters
+    at two CTAs per SM, in clusters of 1, 2, 3, 4, 6, 8, 10, 12 or 16.
+    Batched calls (8-warp CTAs, two tokens per pass on matrices of at most 32
+    MiB of packed planes, else eight) fill the SMs' CTA slots once at most."""
     for M, N, K, g, nS, Ks in ((4096, 4096, 2, 4, 128, 2), (11008, 4096, 2, 4, 123, 2), (8192, 8192, 3, 8, 410, 2)):
         s = fake_weights(M=M, N=N, K=K, g=g, nS=nS, Ks=Ks)
         ind = fb.fb_gemv_launch_plan(s, 1, 3, 148)
@@ -211,7 +212,9 @@ def test_launch_plan_shapes_by_call_kind(L):
         assert ind["warps"] == 8 and ind["cpb"] <= (64 if M * N * K >= 64 * 8 * 2**20 else 32)
         assert dep["warps"] == 8 and dep["cpb"] <= 32 and dep["cpb"] % 8 == 0
         assert dep["C"] * dep["RB"] <= 2 * 148 and dep["C"] in (1, 2, 3, 4, 6, 8, 10, 12, 16)
-        assert bat["warps"] == 8 and bat["C"] * bat["RB"] * 2 <= 2 * 148   # 16 tokens: two passes
+        small = M * N * K <= 32 * 8 * 2**20             # at most 32 MiB of packed planes
+        passes = 8 if small else 2                       # 16 tokens: passes of 2 (three CTAs per SM) or 8
+        assert bat["warps"] == 8 and bat["C"] * bat["RB"] * passes <= (3 if small else 2) * 148
 
 
 def test_launch_plan_rejects_bad_arguments(L):
