@@ -195,8 +195,10 @@ FB_API fb_status fb_gemv(const fb_weights *W, const void *x, fb_dtype t, float *
 
 /* fb_gemv_batched: Y[b*ldy + i] = sum_j W_hat[i][j] * X[b*ldx + j] for
  * b < batch (1 <= batch <= 64), i < M.  ldx >= N, ldy >= M.  The tokens are
- * processed in passes of up to 8: within a pass, each weight word is read
- * from memory once and applied to every token's tables.  Per token the
+ * processed in passes (of 2 tokens for matrices of at most 32 MiB of packed
+ * planes, whose passes share the weights through L2; else of up to 8):
+ * within a pass, each weight word is read from memory once and applied to
+ * every token's tables.  Per token the
  * result has the same properties as fb_gemv's (fp32 sums, deterministic,
  * same tolerance). */
 FB_API fb_status fb_gemv_batched(const fb_weights *W, const void *X, fb_dtype t, int batch, int ldx,
@@ -245,7 +247,8 @@ FB_API fb_status fb_gemv_group_scales(const fb_weights *W, int G, const void *x,
  * FB_PLAN="C,cpb[,n]", read when a plan is first made for a shape, forces the
  * cluster size and row block (clamped to what the matrix and shared memory
  * allow); the optional n is, for batch-1 calls, 16 to use 16-warp CTAs (one
- * per SM) and, for batched calls, the tokens per pass (even, at most 16). */
+ * per SM) and, for batched calls, the tokens per pass (even, at most 16; a
+ * forced plan uses the kernel variant with two CTAs per SM). */
 FB_API fb_status fb_gemv_launch_plan(const fb_weights *W, int batch, unsigned flags, int sms, int *out);
 
 /* fb_device_errors: synchronises the current device, then stores in *flags
