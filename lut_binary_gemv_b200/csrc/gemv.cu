@@ -532,14 +532,14 @@ constexpr int kZBytes = 2 * kPanelCols * 4;
 // ---- The streaming kernel: weights straight into registers --------------
 //
 // The packed weights are not staged in shared memory: each lane loads its
-// rows' words of the panel after next with 128-bit loads into one of two
-// register sets while it looks up the current panel from the other, so a
-// weight byte costs shared-memory bandwidth only for its table lookup.  8
-// warps per CTA and about 70 KB of shared memory let two CTAs share an SM,
-// so one CTA's prologue, barriers and reduction overlap the other's
-// lookups.  For calls that depend on the previous kernel the first two
-// panels' words (and an L2 prefetch of the rest of the slice) are requested
-// before the programmatic-launch wait.
+// rows' words of a later panel with 128-bit loads into registers right
+// after it has looked up the current ones, so a weight byte costs
+// shared-memory bandwidth only for its table lookup.  8 warps per CTA and
+// about 70 KB of shared memory let two or three CTAs share an SM, so one
+// CTA's prologue, barriers and reduction overlap the others' lookups.  For
+// calls that depend on the previous kernel the first panel's words (two
+// panels' for warps of one or two items) and an L2 prefetch of the next
+// panels are requested before the programmatic-launch wait.
 
 // 16 bytes of packed weights, read once: not kept in L1.
 __device__ __forceinline__ uint4 ldg_stream(const void *p) {
@@ -1546,8 +1546,8 @@ static fb_status launch_gemv(const fb_weights *const *Ws, int n, const void *X, 
     attr[0].val.clusterDim.x = pl.C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    // a cluster's CTAs on different SMs: two CTAs of one call sharing an SM
-    // would each run at half speed, and the cluster waits for its slowest
+    // a cluster's CTAs on different SMs where possible: CTAs of one cluster
+    // sharing an SM slow each other, and the cluster waits for its slowest
     attr[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
     attr[1].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicySpread;
     int na = 2;

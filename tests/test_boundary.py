@@ -215,6 +215,9 @@ def test_launch_plan_shapes_by_call_kind(L):
         small = M * N * K <= 32 * 8 * 2**20             # at most 32 MiB of packed planes
         passes = 8 if small else 2                       # 16 tokens: passes of 2 (three CTAs per SM) or 8
         assert bat["warps"] == 8 and bat["C"] * bat["RB"] * passes <= (3 if small else 2) * 148
+        per_sm = 3 if small else 2                       # CTAs that must fit in an SM's 228 KB
+        assert per_sm * (bat["smem"] + 1024) <= 228 * 1024
+        assert 3 * (ind["smem"] + 1024) <= 228 * 1024 or ind["cpb"] > 32   # independent: three per SM
 
 
 def test_launch_plan_rejects_bad_arguments(L):
