@@ -1196,8 +1196,9 @@ int stream_items(int cpb, int nw = kStreamWarps) { return cpb <= nw ? 1 : cpb <=
 // the largest independent calls and with the tuning override -- and
 // clusters of up to 16 CTAs).
 //  * Independent calls overlap their neighbours: row blocks of 32 chunks
-//    (few table builds per row), C = 2 for matrices of at most 8 row
-//    blocks, else 1.
+//    (few table builds per row; 64 from 64 MiB of packed planes), small
+//    clusters (1 for at most 4 row blocks and 40 virtual panels, 2 for at
+//    most 8 row blocks, else 1).
 //  * A call that waits for its predecessor: the plan of least modelled
 //    latency (per panel a CTA works through, a fixed cost and a cost per
 //    chunk of rows; times the waves of clusters that fit at two CTAs per
@@ -1225,9 +1226,12 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         // Matrices of at least 64 MiB of packed planes (65536 items): row
         // blocks of 64 chunks (eight per warp) in clusters of 2 -- the
         // fewest table builds per row.  Smaller ones: row blocks of up to 32
-        // chunks, C = 2 for matrices of at most 8 row blocks, else 1 (on
-        // those, 64-chunk blocks make each CTA live so long that graphs of
-        // such calls lose more to filling and draining than they gain).
+        // chunks, C = 1 for matrices of at most 4 row blocks and 40 virtual
+        // panels (4096^2: no cluster reduction; 1.377 -> 1.365 us, the
+        // 7B-shaped step 0.643 -> 0.613 ms), else C = 2 for at most 8 row
+        // blocks (a CTA's panel list stays short), else 1 (on those, 64-chunk
+        // blocks make each CTA live so long that graphs of such calls lose
+        // more to filling and draining than they gain).
         // Measured on B200 in graphs of independent calls: 28672x8192 and
         // 8192x28672 with K = 3 run 12-13% faster with 64-chunk blocks,
         // 8192^2 K = 3 9% slower, 4096^2 (the 7B-shaped matrices) slower
@@ -1239,7 +1243,7 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
             set(2, 2 * max_cpb);
         } else {
             const int RB = ceil_div(pl.nchunks, max_cpb);
-            set(RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
+            set(RB <= 4 && pl.V <= 40 ? 1 : RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
         }
     } else {
         // Latency model of a call that waits for its predecessor (fitted to
