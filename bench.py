@@ -404,18 +404,19 @@ def run_ours(args):
     # e2e through the public API, every step: the step's x copied in from
     # pinned host memory, its 64 fb_gemv calls (independent calls, replayed
     # from a captured CUDA graph), its y read back into pinned host memory.
-    # Steps are double-buffered: step k's copies and GEMVs run on their own
-    # streams (host-to-device, compute k % 2, device-to-host), so they
+    # Steps rotate through three buffer sets: step k's copies and GEMVs run
+    # on their own streams (host-to-device, compute k % 3, device-to-host), so they
     # overlap the neighbouring steps' work; events keep each buffer's copy in
     # -> GEMVs -> copy out order.  The timed region spans the first step's
     # copy in to the last step's copy out.  The same with 64 eager Python
     # calls per step on one stream, not overlapped, is reported beside it.
     n_e2e = WEIGHT_SETS
     x_host = torch.stack([x.cpu() for x in xs]).pin_memory()
-    y_hosts = [torch.empty((n_e2e, 4096), dtype=torch.float32).pin_memory() for _ in range(2)]
+    NBUF = 3   # buffer sets (and compute streams) the steps rotate through
+    y_hosts = [torch.empty((n_e2e, 4096), dtype=torch.float32).pin_memory() for _ in range(NBUF)]
     y_host = y_hosts[0]
-    x_devs = [torch.empty_like(x_host, device=device) for _ in range(2)]
-    y_devs = [torch.empty((n_e2e, 4096), dtype=torch.float32, device=device) for _ in range(2)]
+    x_devs = [torch.empty_like(x_host, device=device) for _ in range(NBUF)]
+    y_devs = [torch.empty((n_e2e, 4096), dtype=torch.float32, device=device) for _ in range(NBUF)]
     x_dev, y_dev = x_devs[0], y_devs[0]
     e2e_steps = max(10, args.steps // 10)
 
@@ -439,16 +440,16 @@ def run_ours(args):
             for r in range(n_e2e):
                 fb.fb_gemv(Ws[r], x_devs[b][r], y=y_devs[b][r], flags=indep)
         return body
-    g_e2e = [capture(stream, gemvs_e2e(b)) for b in range(2)]
+    g_e2e = [capture(stream, gemvs_e2e(b)) for b in range(NBUF)]
     h2d, d2h = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
-    comp = [torch.cuda.Stream(device=device) for _ in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    comp = [torch.cuda.Stream(device=device) for _ in range(NBUF)]
+    ev_in = [torch.cuda.Event() for _ in range(NBUF)]
+    ev_comp = [torch.cuda.Event() for _ in range(NBUF)]
+    ev_out = [torch.cuda.Event() for _ in range(NBUF)]
 
     def e2e_pipelined(steps):
         for _ in range(3):   # warm-up, one buffer at a time
-            for b in range(2):
+            for b in range(NBUF):
                 x_devs[b].copy_(x_host, non_blocking=True)
                 g_e2e[b].replay()
                 y_hosts[b].copy_(y_devs[b], non_blocking=True)
@@ -459,14 +460,14 @@ def run_ours(args):
         for st in (d2h, *comp):
             st.wait_event(s0)
         for k in range(steps):
-            b = k % 2
+            b = k % NBUF
             with torch.cuda.stream(h2d):
-                h2d.wait_event(ev_comp[b])          # step k - 2 has finished reading x_devs[b]
+                h2d.wait_event(ev_comp[b])          # step k - NBUF has finished reading x_devs[b]
                 x_devs[b].copy_(x_host, non_blocking=True)
                 ev_in[b].record(h2d)
             with torch.cuda.stream(comp[b]):
                 comp[b].wait_event(ev_in[b])
-                comp[b].wait_event(ev_out[b])       # step k - 2's y has left y_devs[b]
+                comp[b].wait_event(ev_out[b])       # step k - NBUF's y has left y_devs[b]
                 g_e2e[b].replay()
                 ev_comp[b].record(comp[b])
             with torch.cuda.stream(d2h):
@@ -526,8 +527,8 @@ def run_ours(args):
                 "d2h_bytes_per_step": int(y_host.numel() * 4),
                 "note": (f"per step: pinned host x ({n_e2e} x 4096 fp16) copied in, {n_e2e} fb_gemv calls "
                          "(PDL + FB_GEMV_INDEPENDENT, replayed from a CUDA graph), y read back to pinned host; "
-                         "steps double-buffered on their own streams, so one step's copies overlap its "
-                         "neighbours' GEMVs")},
+                         "steps rotate through three buffer sets on their own streams, so one step's copies "
+                         "overlap its neighbours' GEMVs")},
         "e2e_eager": {"value": round(e2e_eager_gbs, 2), "unit": "GB/s",
                       "note": f"the same with {n_e2e} eager Python fb_gemv calls per step (dependent-call plan)"},
         "gpu_launches": args.steps * gemvs,
