@@ -102,7 +102,14 @@ def _check(status: int, what: str):
         raise FbError(status, what)
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device) -> int:
+    """The current CUDA stream of `device` as a raw handle (the cheap
+    accessor when torch has it: eager calls are bound by host time)."""
+    if _raw_stream is not None:
+        return _raw_stream(device.index if device.index is not None else torch.cuda.current_device())
     return torch.cuda.current_stream(device).cuda_stream
 
 
@@ -196,7 +203,10 @@ class Weights:
 
     @property
     def ref(self):
-        return C.byref(self.struct)
+        ref = self.__dict__.get("_ref")
+        if ref is None:
+            ref = self._ref = C.byref(self.struct)
+        return ref
 
     def with_g(self, g: int) -> "Weights":
         """The same tensors with another LUT group width (the packed layout
@@ -260,9 +270,10 @@ def fb_gemv(W: Weights, x: torch.Tensor, y: Optional[torch.Tensor] = None,
     if x.stride(-1) != 1:
         x = x.contiguous()
     y = torch.empty(W.M, dtype=torch.float32, device=x.device) if y is None else y
-    ws = W.workspace(1) if ws is None else ws
-    _check(lib().fb_gemv(W.ref, x.data_ptr(), _DTYPES[x.dtype], y.data_ptr(), ws.data_ptr(),
-                         ws.numel() * ws.element_size(), flags, _stream(x.device)), "fb_gemv")
+    # the kernels need no workspace (fb_gemv_workspace_bytes is 0): NULL, 0 unless one is given
+    wp, wn = (None, 0) if ws is None else (ws.data_ptr(), ws.numel() * ws.element_size())
+    _check(lib().fb_gemv(W.ref, x.data_ptr(), _DTYPES[x.dtype], y.data_ptr(), wp, wn, flags,
+                         _stream(x.device)), "fb_gemv")
     return y
 
 
@@ -273,10 +284,9 @@ def fb_gemv_batched(W: Weights, X: torch.Tensor, Y: Optional[torch.Tensor] = Non
     if X.stride(-1) != 1:
         X = X.contiguous()
     Y = torch.empty((B, W.M), dtype=torch.float32, device=X.device) if Y is None else Y
-    ws = W.workspace(B) if ws is None else ws
+    wp, wn = (None, 0) if ws is None else (ws.data_ptr(), ws.numel() * ws.element_size())
     _check(lib().fb_gemv_batched(W.ref, X.data_ptr(), _DTYPES[X.dtype], B, X.stride(0), Y.data_ptr(),
-                                 Y.stride(0), ws.data_ptr(), ws.numel() * ws.element_size(), flags,
-                                 _stream(X.device)), "fb_gemv_batched")
+                                 Y.stride(0), wp, wn, flags, _stream(X.device)), "fb_gemv_batched")
     return Y
 
 
