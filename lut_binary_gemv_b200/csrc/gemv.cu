@@ -1197,8 +1197,8 @@ int stream_items(int cpb, int nw = kStreamWarps) { return cpb <= nw ? 1 : cpb <=
 // clusters of up to 16 CTAs).
 //  * Independent calls overlap their neighbours: row blocks of 32 chunks
 //    (few table builds per row; 64 from 64 MiB of packed planes), small
-//    clusters (1 for at most 4 row blocks and 40 virtual panels, 2 for at
-//    most 8 row blocks, else 1).
+//    clusters (for at most 4 row blocks one CTA per ~24 virtual panels,
+//    1 up to 40; 2 for at most 8 row blocks; else 1).
 //  * A call that waits for its predecessor: the plan of least modelled
 //    latency (per panel a CTA works through, a fixed cost and a cost per
 //    chunk of rows; times the waves of clusters that fit at two CTAs per
@@ -1217,7 +1217,7 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
     pl.kind = 1;
     const int max_cpb = 4 * kStreamWarps;   // default plans: up to 4 items per warp
     auto set = [&](int C, int cpb) {
-        pl.C = std::min(C, pl.V);
+        pl.C = std::max(1, std::min(std::min(C, pl.V), kMaxCluster));   // (vsplit holds kMaxCluster + 1 cuts)
         pl.cpb = std::min(cpb, pl.nchunks);
         pl.RB = ceil_div(pl.nchunks, pl.cpb);
         split_weighted(groups, pl.C, pl.cpb, pl.vsplit);
@@ -1226,12 +1226,15 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         // Matrices of at least 64 MiB of packed planes (65536 items): row
         // blocks of 64 chunks (eight per warp) in clusters of 2 -- the
         // fewest table builds per row.  Smaller ones: row blocks of up to 32
-        // chunks, C = 1 for matrices of at most 4 row blocks and 40 virtual
-        // panels (4096^2: no cluster reduction; 1.377 -> 1.365 us, the
-        // 7B-shaped step 0.643 -> 0.613 ms), else C = 2 for at most 8 row
-        // blocks (a CTA's panel list stays short), else 1 (on those, 64-chunk
-        // blocks make each CTA live so long that graphs of such calls lose
-        // more to filling and draining than they gain).
+        // chunks; matrices of at most 4 row blocks take C = 1 up to 40
+        // virtual panels (4096^2: no cluster reduction; 1.377 -> 1.365 us,
+        // the 7B-shaped step 0.643 -> 0.613 ms) and about 24 panels per CTA
+        // beyond (4096x11008, 90 panels: C = 4; 4.63 -> 4.04 us, the step
+        // 0.613 -> 0.587 ms); C = 2 for at most 8 row blocks, else 1 (on
+        // those, 64-chunk blocks make each CTA live so long that graphs of
+        // such calls lose more to filling and draining than they gain; C = 2
+        // on the 11 row blocks of 11008x4096 was faster alone but slower in
+        // the 7B-shaped step).
         // Measured on B200 in graphs of independent calls: 28672x8192 and
         // 8192x28672 with K = 3 run 12-13% faster with 64-chunk blocks,
         // 8192^2 K = 3 9% slower, 4096^2 (the 7B-shaped matrices) slower
@@ -1243,7 +1246,8 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
             set(2, 2 * max_cpb);
         } else {
             const int RB = ceil_div(pl.nchunks, max_cpb);
-            set(RB <= 4 && pl.V <= 40 ? 1 : RB <= 8 ? 2 : 1, ceil_div(pl.nchunks, RB));
+            set(RB <= 4 ? (pl.V <= 40 ? 1 : std::min(kMaxCluster, std::max(2, (pl.V + 12) / 24))) : RB <= 8 ? 2 : 1,
+                ceil_div(pl.nchunks, RB));
         }
     } else {
         // Latency model of a call that waits for its predecessor (fitted to
