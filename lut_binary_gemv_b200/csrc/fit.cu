@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kFitMaxSweeps = 1000;
 constexpr int kSelectThreads = 1024;
-constexpr int kRowUnroll = 4;     // float4s a lane loads per row before adding them (row pass)
+constexpr int kRowUnroll = 8;     // float4s a lane loads per row before adding them (row pass)
 constexpr int kColSplit = 16;     // CTAs of a column-pass cluster: slices of the rows
 constexpr int kColTile = 128;     // columns of a column-pass CTA: a float4 per lane
 constexpr int kColUnroll = 8;     // rows a warp loads before adding them (column passes)
