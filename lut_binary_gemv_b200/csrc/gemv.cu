@@ -1230,7 +1230,9 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
         // virtual panels (4096^2: no cluster reduction; 1.377 -> 1.365 us,
         // the 7B-shaped step 0.643 -> 0.613 ms) and about 24 panels per CTA
         // beyond (4096x11008, 90 panels: C = 4; 4.63 -> 4.04 us, the step
-        // 0.613 -> 0.587 ms); C = 2 for at most 8 row blocks, else 1 (on
+        // 0.613 -> 0.587 ms; with group-wise row scales of 128 columns,
+        // whose half-panels double the panel count, C = 2: 2.88 -> 2.78 us
+        // at 4096^2); C = 2 for at most 8 row blocks, else 1 (on
         // those, 64-chunk blocks make each CTA live so long that graphs of
         // such calls lose more to filling and draining than they gain; C = 2
         // on the 11 row blocks of 11008x4096 was faster alone but slower in
@@ -1246,7 +1248,8 @@ Plan make_stream_plan(const fb_weights *W, int batch, int sms, bool independent,
             set(2, 2 * max_cpb);
         } else {
             const int RB = ceil_div(pl.nchunks, max_cpb);
-            set(RB <= 4 ? (pl.V <= 40 ? 1 : std::min(kMaxCluster, std::max(2, (pl.V + 12) / 24))) : RB <= 8 ? 2 : 1,
+            set(RB <= 4 ? (pl.V <= 40 ? 1 : G == 128 ? 2 : std::min(kMaxCluster, std::max(2, (pl.V + 12) / 24)))
+                        : RB <= 8 ? 2 : 1,
                 ceil_div(pl.nchunks, RB));
         }
     } else {
