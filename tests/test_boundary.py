@@ -220,6 +220,22 @@ def test_launch_plan_shapes_by_call_kind(L):
         assert 3 * (ind["smem"] + 1024) <= 228 * 1024 or ind["cpb"] > 32   # independent: three per SM
 
 
+def test_independent_plans_keep_a_ctas_panel_list_short(L):
+    """Calls flagged independent on matrices of at most 4 row blocks split
+    the virtual panels so that a CTA works through at most 40 of them (one
+    CTA per row block up to 40 panels, about 24 per CTA beyond); larger
+    matrices keep row blocks of 32 or 64 chunks in clusters of 1 or 2."""
+    for M, N, K, g, nS, Ks in ((4096, 4096, 2, 4, 128, 2), (4096, 11008, 2, 4, 330, 2), (1024, 28672, 3, 8, 1434, 2),
+                               (4096, 65536, 1, 2, 0, 2), (11008, 4096, 2, 4, 123, 2), (8192, 8192, 3, 8, 410, 2)):
+        s = fake_weights(M=M, N=N, K=K, g=g, nS=nS, Ks=Ks)
+        plan = fb.fb_gemv_launch_plan(s, 1, 3, 148)
+        if plan["RB"] <= 4 and plan["cpb"] <= 32:
+            assert -(-plan["V"] // plan["C"]) <= 40 or plan["C"] == 16
+            assert plan["C"] == 1 or plan["V"] > 40
+        else:
+            assert plan["C"] <= 2
+
+
 def test_launch_plan_rejects_bad_arguments(L):
     s = fake_weights()
     out = (C.c_int * 6)()
