@@ -39,7 +39,7 @@ def _rank_main(rank, world, port, values, out):
 def test_max_over_ranks_with_gloo():
     world, port = 2, free_port()
     values = [3.25, 7.5]
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(world, port, values, out), nprocs=world, join=True)
         assert dict(out) == {0: 7.5, 1: 7.5}
