@@ -197,6 +197,28 @@ def test_launch_plan_fits_at_the_abi_corners(L, M, N, K, nS, Ks, batch, flags):
     assert plan["RB"] * plan["cpb"] >= nchunks > (plan["RB"] - 1) * plan["cpb"]
 
 
+def test_launch_plan_fits_on_random_valid_arguments(L):
+    """Seeded sweep over valid sizes, salient counts, batches, flags and SM
+    counts (1 to 296): every plan fits one CTA's shared memory and covers the
+    matrix."""
+    import random
+    rng = random.Random(7)
+    seen = 0
+    while seen < 3000:
+        M = rng.choice([1, 31, 33, 4096, 11008, 131077, 1 << 24, rng.randint(1, 300000)])
+        N = rng.choice([32, 96, 288, 4096, 11008, 28672, 1 << 20, 32 * rng.randint(1, 20000)])
+        g = rng.choice([1, 2, 4, 8])
+        nS = min(N, rng.choice([0, 0, 1, 31, 33, N // 20, N]))
+        s = fake_weights(M=M, N=N, K=rng.randint(1, 4), g=g, nS=nS, Ks=rng.randint(1, 4))
+        batch, flags = rng.choice([1, 2, 3, 16, 17, 64]), rng.choice([0, 1, 2, 3])
+        plan = fb.fb_gemv_launch_plan(s, batch, flags, rng.choice([1, 2, 16, 132, 148, 296]))
+        nchunks = -(-M // 32)
+        assert 0 < plan["smem"] <= 225 * 1024, (M, N, nS, batch, flags, plan)
+        assert 1 <= plan["C"] <= min(16, plan["V"]) and plan["RB"] <= 65535, (M, N, nS, batch, flags, plan)
+        assert plan["RB"] * plan["cpb"] >= nchunks > (plan["RB"] - 1) * plan["cpb"]
+        seen += 1
+
+
 def test_launch_plan_shapes_by_call_kind(L):
     """Batch-1 calls get the 8-warp streaming CTA with rows in whole chunks
     per warp; calls flagged independent take row blocks of up to 32 chunks
