@@ -151,6 +151,10 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert L.fb_vcm_gather(FAKE, 1, 1, 64, 64, None, 10, 32, FAKE, 32, None) == INVALID
     assert L.fb_validate_weights(C.byref(fake_weights(g=5))) == INVALID
     assert L.fb_validate_weights(None) == INVALID
+    s = fake_weights(M=64, N=512)
+    for G in (64, 192, 384, 1024, 0, -128):     # not 128, N or a multiple of 256 dividing N
+        assert L.fb_gemv_group_scales(C.byref(s), G, FAKE, 0, FAKE, 0, None) == INVALID
+    assert L.fb_gemv_group_scales(C.byref(fake_weights(K=5)), 128, FAKE, 0, FAKE, 0, None) == INVALID
 
 
 @pytest.mark.parametrize("shape", [
