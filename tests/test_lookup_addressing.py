@@ -114,3 +114,28 @@ def test_repeated_narrow_columns_cover_the_copies():
                 assert slot_group < copies * Bp
             else:
                 assert slot_group >= copies * Bp
+
+
+def z_slot(t):
+    """Slot of panel column t in the z buffer: the low four columns of each
+    8-column group first (group q at 4q), the high four after them (128 + 4q)."""
+    return (128 if t & 4 else 0) + 4 * (t >> 3) + (t & 3)
+
+
+def test_z_layout_gives_contiguous_build_reads():
+    """The table build's lane q reads its group's z as two 16-byte words at
+    4q and 128 + 4q: they must hold columns 8q..8q+3 and 8q+4..8q+7 in order,
+    and a warp's 32 words must be consecutive (4 wavefronts per read).  The
+    z stores (thread t writes column t) then hit each bank twice: one extra
+    wavefront per warp and panel, the price of the contiguous reads."""
+    assert sorted(z_slot(t) for t in range(256)) == list(range(256))
+    inv = {z_slot(t): t for t in range(256)}
+    for q in range(32):
+        assert [inv[4 * q + i] for i in range(4)] == [8 * q + i for i in range(4)]
+        assert [inv[128 + 4 * q + i] for i in range(4)] == [8 * q + 4 + i for i in range(4)]
+    for base in (0, 128):
+        words = [base + 4 * q for q in range(32)]
+        assert words == list(range(base, base + 128, 4))                  # 512 consecutive bytes
+    for w in range(8):
+        banks = [z_slot(32 * w + i) % 32 for i in range(32)]
+        assert max(banks.count(b) for b in set(banks)) == 2
