@@ -233,6 +233,7 @@ def test_sampled_rows_match_full():
     np.testing.assert_array_equal(oracle.gemv_lut(w, 4, x, rows), oracle.gemv_lut(w, 4, x)[:, rows])
     for b in range(3):   # batch rows are independent problems
         np.testing.assert_array_equal(oracle.gemv(w, x[b])[0][0], y[b])
+        np.testing.assert_array_equal(oracle.gemv_lut(w, 4, x[b])[0], oracle.gemv_lut(w, 4, x)[b])
 
 
 # --- invariants ---------------------------------------------------------------
@@ -248,6 +249,27 @@ def test_salient_over_all_columns_equals_extra_global_bases():
                               np.concatenate([p.alpha_c, p.s_alpha_c]))
     y2, _, _ = oracle.gemv(w2, oracle.x_to_f64(p.x, p.x_dtype))
     assert np.array_equal(y, y2)
+
+
+def test_negating_a_base_and_its_scale_changes_nothing():
+    """(-alpha_r) alpha_c^T (.) (-B) is the same term: flipping every sign of
+    a base (global or salient) and negating its row scales leaves W, y and
+    both tolerance magnitudes d and e unchanged (e sums |alpha_r alpha_c x|)."""
+    p = wl.make_problem(40, 128, 3, nS=17, Ks=2, x_dtype="f32", seed=27, batch=2)
+    x = oracle.x_to_f64(p.x, p.x_dtype)
+    W0 = oracle.dequant(oracle.OracleWeights.from_problem(p))
+    y0, d0, e0 = oracle.problem_reference(p)
+    signs, s_signs = p.signs(), p.s_signs()
+    signs[1] *= -1
+    s_signs[0] *= -1
+    ar, s_ar = p.alpha_r.copy(), p.s_alpha_r.copy()
+    ar[1] *= -1
+    s_ar[0] *= -1
+    w = _weights_from_signs(signs, ar, p.alpha_c, p.s_idx, s_signs, s_ar, p.s_alpha_c)
+    assert np.array_equal(oracle.dequant(w), W0)
+    y, d, e = oracle.gemv(w, x)
+    assert np.array_equal(y, y0) and np.array_equal(d, d0) and np.array_equal(e, e0)
+    assert np.array_equal(oracle.gemv_lut(w, 4, x), oracle.gemv_lut(oracle.OracleWeights.from_problem(p), 4, x))
 
 
 def test_empty_salient_equals_global_term():

@@ -4,6 +4,11 @@ Each mutation edits one expression of ``oracle/oracle.c`` (a sign, a bit
 order, an index, a dropped term), compiles the edited copy into a temporary
 library, and runs ``tests/test_oracle.py`` against it in a subprocess.  The
 pins must reject every mutant.  The real oracle is never modified.
+
+Edits that cannot change any result are not listed: the salient padding is
+zeroed twice (x and alpha_c past nS are both 0), so giving it alpha_c = 1 or a
+set pattern bit changes nothing, and e takes fabs of a whole product, so
+dropping the fabs of its row scale changes nothing either.
 """
 
 import os
@@ -33,6 +38,20 @@ MUTATIONS = [
     ("last column dropped", "acc += Wrow[j] * xb[j];", "if (j + 1 < N) acc += Wrow[j] * xb[j];"),
     ("tolerance magnitude signed", "mag += fabs(Wrow[j] * xb[j]);", "mag += Wrow[j] * xb[j];"),
     ("salient x gather", "x_S[t] = x[s_idx[t]];", "x_S[t] = x[t];"),
+    ("e: salient bases dropped", "m2 += fabs(ar * w->s_alpha_c[(size_t)k * w->nS + t] * xb[w->s_idx[t]]);",
+     "m2 += 0.0 * fabs(ar * w->s_alpha_c[(size_t)k * w->nS + t] * xb[w->s_idx[t]]);"),
+    ("e: salient x not gathered", "* xb[w->s_idx[t]]);", "* xb[t]);"),
+    ("e: global alpha_c dropped", "m2 += fabs(ar * ac * xb[j]);", "m2 += fabs(ar * xb[j]);"),
+    ("fp16 subnormal scale", "ldexp((double)m, -24)", "ldexp((double)m, -25)"),
+    ("bf16 decode shift", "(uint32_t)b << 16", "(uint32_t)b << 15"),
+    ("dense batch stride", "const double *xb = x + (size_t)b * N;\n                double acc",
+     "const double *xb = x;\n                double acc"),
+    ("LUT batch stride", "const double *xb = x + (size_t)b * N;\n        lut_tables",
+     "const double *xb = x;\n        lut_tables"),
+    ("salient alpha_c of base 0", "s_alpha_c[(size_t)k * w->nS + t];\n            Wrow", "s_alpha_c[t];\n            Wrow"),
+    ("salient alpha_r of base 0", "const double ar = w->s_alpha_r[(size_t)k * M + i];\n        for (int64_t t",
+     "const double ar = w->s_alpha_r[i];\n        for (int64_t t"),
+    ("LUT alpha_r of base 0", "acc += w->alpha_r[(size_t)k * M + i] * s;", "acc += w->alpha_r[i] * s;"),
 ]
 
 
