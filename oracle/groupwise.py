@@ -1,8 +1,8 @@
 """fp64 CPU oracle for group-wise row scales (the "g128" format variant).
 
-TEST INFRASTRUCTURE ONLY: only tests/ may import this module (there is no
-GPU kernel for this variant yet).  The library never imports it, and it
-imports nothing from the library.
+TEST INFRASTRUCTURE ONLY: only tests/ may import this module (the GPU
+variant, fb_gemv_group_scales, is checked against it there).  The library
+never imports it, and it imports nothing from the library.
 
 The FluxBin page (Experimental results, the accuracy paragraph) names a
 "2b-s16-g128" setting without defining it.  Reading taken: "g128" is the
