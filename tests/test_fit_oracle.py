@@ -77,6 +77,13 @@ def test_saliency_constructed_cases():
     s = F.saliency_scores(Wc, np.ones((5, 12)))
     assert F.select_salient(s, 4).tolist() == [8, 9, 10, 11]
     np.testing.assert_allclose(s, 5 * 4 * (np.arange(12) + 1.0) ** 2)
+    # equal weight columns: the activation term is the Hessian's diagonal,
+    # diag(X^T X) (a matrix product here), so a single large activation
+    # (3: 9) outranks spread ones (2, 2: 8; 1, 1, 1, 1: 4)
+    Xd = np.array([[3.0, 1.0, 2.0], [0.0, 1.0, 2.0], [0.0, 1.0, 0.0], [0.0, -1.0, 0.0]])
+    sd = F.saliency_scores(np.ones((4, 3)), Xd)
+    np.testing.assert_array_equal(sd, 4 * np.diag(Xd.T @ Xd))
+    assert F.select_salient(sd, 1).tolist() == [0] and F.select_salient(sd, 2).tolist() == [0, 2]
 
 
 def test_select_equal_scores_take_the_lower_column_and_list_ascending():
@@ -150,7 +157,8 @@ def _pins_pass():
         for s in (1, 2, 8):
             test_residual_never_grows(s)
         test_more_bases_and_salient_bases_fit_better()
-    except (AssertionError, ValueError, FloatingPointError):
+        test_fitted_factors_through_the_gemv_oracle()
+    except (AssertionError, ValueError, FloatingPointError, IndexError):
         return False
     return True
 
@@ -171,3 +179,35 @@ def test_planted_mistakes_fail_a_pin(monkeypatch, mutation):
         monkeypatch.setattr(F, "select_salient",   # equal scores take the higher column
                             lambda s, n: np.sort(np.lexsort((-np.arange(len(s)), -np.asarray(s)))[:n]).astype(np.uint32))
     assert not _pins_pass()
+
+
+SOURCE_MUTATIONS = [
+    ("residual update sign", "R_next = R - np.outer(ar, ac) * B", "R_next = R + np.outer(ar, ac) * B"),
+    ("one sweep too few", "for _ in range(sweeps):", "for _ in range(sweeps - 1):"),
+    ("column scale from the old row scale", "        ar = _scaled(A @ ac, _norm2(ac))\n        ac = _scaled(A.T @ ar, _norm2(ar))",
+     "        ac_old = ac\n        ar = _scaled(A @ ac, _norm2(ac))\n        ac = _scaled(A.T @ ar, _norm2(ac_old))"),
+    ("activation energy not squared", 'np.einsum("tj,tj->j", X, X)', 'np.einsum("tj->j", np.abs(X))'),
+    ("weight energy over rows", 'np.einsum("ij,ij->j", W, W)', 'np.einsum("ij,ij->j", W, np.abs(W) ** 0.5)'),
+    ("smallest scores selected", "np.argsort(-score, kind=\"stable\")", "np.argsort(score, kind=\"stable\")"),
+    ("salient set not listed ascending", "return np.sort(order[:nS]).astype(np.uint32)",
+     "return order[:nS].astype(np.uint32)"),
+    ("salient residual not written back", "        R[:, S.astype(np.int64)] = RS\n", ""),
+    ("salient bases fitted before the global ones", "    for k in range(K):\n        signs[k], alpha_r[k], alpha_c[k], R = fit_base(R, sweeps)\n",
+     ""),
+]
+
+
+@pytest.mark.parametrize("name,old,new", SOURCE_MUTATIONS, ids=[m[0] for m in SOURCE_MUTATIONS])
+def test_planted_source_mistakes_fail_a_pin(monkeypatch, name, old, new):
+    """Each edits one step of a copy of ``oracle/fit.py`` (loaded as a new
+    module; the real one is untouched) and the pins, run against the copy,
+    must fail."""
+    import sys
+    import types
+    src = open(F.__file__).read()
+    assert src.count(old) == 1, name
+    mod = types.ModuleType("fit_mutant")
+    mod.__file__ = F.__file__
+    exec(compile(src.replace(old, new), F.__file__, "exec"), mod.__dict__)
+    monkeypatch.setattr(sys.modules[__name__], "F", mod)
+    assert not _pins_pass(), name
