@@ -86,3 +86,35 @@ def test_planted_group_index_mistake_fails(monkeypatch):
         test_each_group_is_the_ordinary_format_on_its_columns()
     with pytest.raises(AssertionError):
         test_hand_sized_case_by_loops()
+
+
+SOURCE_MUTATIONS = [
+    ("groups in reverse order", "np.asarray(alpha_r, np.float64)[:, :, grp]", "np.asarray(alpha_r, np.float64)[:, :, grp[::-1]]"),
+    ("column scales ignored", "ac = np.ones((K, N)) if alpha_c is None else np.asarray(alpha_c, np.float64)",
+     "ac = np.ones((K, N))"),
+    ("salient term dropped", "W[:, S] += Ws", "W[:, S] += 0.0 * Ws"),
+    ("salient term on the compact columns", "W[:, S] += Ws", "W[:, :nS] += Ws"),
+    ("row scales of base 0 for every base", "ar = np.asarray(alpha_r, np.float64)[:, :, grp]",
+     "ar = np.asarray(alpha_r, np.float64)[[0] * K][:, :, grp]"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", SOURCE_MUTATIONS, ids=[m[0] for m in SOURCE_MUTATIONS])
+def test_planted_source_mistakes_fail_a_pin(monkeypatch, name, old, new):
+    """Each edits one step of a copy of ``oracle/groupwise.py`` (loaded as a
+    new module; the real one is untouched); one of the pins must fail."""
+    import sys
+    import types
+    src = open(GW.__file__).read()
+    assert src.count(old) == 1, name
+    mod = types.ModuleType("groupwise_mutant")
+    exec(compile(src.replace(old, new), GW.__file__, "exec"), mod.__dict__)
+    monkeypatch.setattr(sys.modules[__name__], "GW", mod)
+    failed = 0
+    for pin in (lambda: test_one_group_is_the_ordinary_format(37), test_each_group_is_the_ordinary_format_on_its_columns,
+                test_hand_sized_case_by_loops):
+        try:
+            pin()
+        except (AssertionError, IndexError, ValueError):
+            failed += 1
+    assert failed, name
