@@ -227,7 +227,7 @@ def cpu_baseline(seconds):
     finally:
         oracle.set_num_threads(cores)
     return {"value": round(p.algorithmic_bytes() / per / 1e9, 4), "unit": "GB/s", "cores": cores,
-            "kind": "oracle", "sample": f"{n} full 4096x4096 K=2 GEMVs (all rows) of the same workload, "
+            "affinity_cpus": len(os.sched_getaffinity(0)), "kind": "oracle", "sample": f"{n} full 4096x4096 K=2 GEMVs (all rows) of the same workload, "
             f"{per * 1e3:.1f} ms each", "ms_per_gemv": round(per * 1e3, 3),
             "single_core": {"value": round(p.algorithmic_bytes() / per1 / 1e9, 4), "unit": "GB/s", "cores": 1,
                             "ms_per_gemv": round(per1 * 1e3, 3),
@@ -265,8 +265,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(),
-            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                             "affinity_cpus": len(os.sched_getaffinity(0)), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
