@@ -568,6 +568,7 @@ def bench_7b(args, device, stream, world, peak):
     steps = max(30, args.steps // 4)
     per = run(fb.FB_GEMV_PDL | fb.FB_GEMV_INDEPENDENT, steps)
     per_dep = run(fb.FB_GEMV_PDL, steps)
+    per_plain = run(0, steps)               # ordinary launches: no programmatic dependent launch
     gbs = total / (per * 1e-3) / 1e9
 
     # Grouped: per layer q,k,v in one launch, o, gate,up in one launch, down
@@ -594,8 +595,11 @@ def bench_7b(args, device, stream, world, peak):
     return {"ms": round(per, 5), "gbs": round(gbs, 2), "frac": round(gbs / peak, 4),
             "ms_dependent_chain": round(per_dep, 5),
             "frac_dependent_chain": round(total / (per_dep * 1e-3) / 1e9 / peak, 4),
+            "ms_plain_chain": round(per_plain, 5),
+            "frac_plain_chain": round(total / (per_plain * 1e-3) / 1e9 / peak, 4),
             "algorithmic_bytes": total, "gemvs": len(Ws), "steps": steps,
-            "note": "224 GEMVs, fresh x per GEMV (independent); dependent chain: each waits for its predecessor",
+            "note": "224 GEMVs, fresh x per GEMV (independent); dependent chain: each waits for its predecessor "
+                    "(programmatic dependent launch); plain chain: the same with ordinary launches",
             "grouped": {"ms": round(per_g, 5), "frac": round(total_g / (per_g * 1e-3) / 1e9 / peak, 4),
                         "ms_dependent_chain": round(per_g_dep, 5),
                         "frac_dependent_chain": round(total_g / (per_g_dep * 1e-3) / 1e9 / peak, 4),

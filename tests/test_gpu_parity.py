@@ -256,6 +256,36 @@ def test_independent_chain_in_graph_matches():
         check(p, y.cpu().numpy()[None].astype(np.float64))
 
 
+def test_plain_and_pdl_graphs_give_the_same_bits():
+    """A graph of ordinary launches (flags 0) and one with programmatic
+    dependent launch compute the same bits for a chain of mixed shapes."""
+    ps = [wl.make_problem(M, N, 2, nS=nS, Ks=2, x_dtype="f16", seed=40 + i)
+          for i, (M, N, nS) in enumerate(((512, 1024, 31), (1100, 512, 16), (256, 2304, 70)))]
+    Ws = [fb.Weights.from_problem(p) for p in ps]
+    xs = [x_tensor(p)[0] for p in ps]
+    s = torch.cuda.Stream()
+    outs = []
+    for flags in (0, fb.FB_GEMV_PDL):
+        ys = [torch.full((p.M,), float("nan"), device=DEV) for p in ps]
+        with torch.cuda.stream(s):
+            for W, x, y in zip(Ws, xs, ys):
+                fb.fb_gemv(W, x, y=y, flags=flags)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(2):
+                    for W, x, y in zip(Ws, xs, ys):
+                        fb.fb_gemv(W, x, y=y, flags=flags)
+        for y in ys:
+            y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        outs.append([y.cpu().numpy() for y in ys])
+    for p, a, b in zip(ps, *outs):
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+        check(p, a[None].astype(np.float64))
+
+
 def test_gemv_in_cuda_graph():
     p = wl.make_problem(1000, 2048, 2, nS=60, Ks=2, x_dtype="f16", seed=11)
     W = fb.Weights.from_problem(p)
