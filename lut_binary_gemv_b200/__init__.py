@@ -195,7 +195,6 @@ class Weights:
         self.planes, self.alpha_r, self.alpha_c = planes, alpha_r, alpha_c
         self.s_idx, self.s_planes, self.s_alpha_r, self.s_alpha_c = s_idx, s_planes, s_alpha_r, s_alpha_c
         self.device = planes.device
-        self._ws = {}
         self.struct = FbWeightsStruct(
             M=M, N=N, K=K, g=g, planes=_ptr(planes), alpha_r=_ptr(alpha_r), alpha_c=_ptr(alpha_c),
             nS=nS, Ks=self.Ks, s_idx=_ptr(s_idx) if nS else None, s_planes=_ptr(s_planes) if nS else None,
@@ -245,15 +244,6 @@ class Weights:
         return cls.from_arrays(p.M, p.N, p.K, p.g if g is None else g, p.sign_bits, p.alpha_r, p.alpha_c,
                                p.s_idx if p.nS else None, p.s_sign_bits, p.s_alpha_r, p.s_alpha_c,
                                device=device)
-
-    def workspace(self, batch: int = 1) -> torch.Tensor:
-        """A zero-filled workspace for this weight set (cached per batch size)."""
-        ws = self._ws.get(batch)
-        if ws is None:
-            n = fb_gemv_workspace_bytes(self, batch)
-            ws = torch.zeros(max(n, 16), dtype=torch.uint8, device=self.device)
-            self._ws[batch] = ws
-        return ws
 
 
 def fb_validate_weights(W: Weights) -> int:
