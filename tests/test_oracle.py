@@ -231,6 +231,7 @@ def test_sampled_rows_match_full():
     np.testing.assert_array_equal(ys, y[:, rows])
     np.testing.assert_array_equal(ds, d[:, rows])
     np.testing.assert_array_equal(oracle.gemv_lut(w, 4, x, rows), oracle.gemv_lut(w, 4, x)[:, rows])
+    np.testing.assert_array_equal(oracle.dequant(w, rows), oracle.dequant(w)[rows])
     for b in range(3):   # batch rows are independent problems
         np.testing.assert_array_equal(oracle.gemv(w, x[b])[0][0], y[b])
         np.testing.assert_array_equal(oracle.gemv_lut(w, 4, x[b])[0], oracle.gemv_lut(w, 4, x)[b])
@@ -337,6 +338,12 @@ def test_rejects_bad_arguments():
         oracle.gemv_lut(oracle.OracleWeights.from_problem(p), 3, np.zeros(32))
     with pytest.raises(ValueError):
         oracle.gemv(oracle.OracleWeights.from_problem(p), np.zeros(32), rows=[8])
+    # more salient columns than columns (each index in range)
+    many = oracle.OracleWeights(8, 32, 1, p.sign_bits, p.alpha_r, p.alpha_c, np.arange(33, dtype=np.uint32) % 32,
+                                np.zeros((1, 8, 8), np.uint8), np.ones((1, 8), np.float32),
+                                np.ones((1, 33), np.float32), 1)
+    with pytest.raises(ValueError):
+        oracle.gemv(many, np.zeros(32))
 
 
 def test_integer_mode_stays_below_2_24():

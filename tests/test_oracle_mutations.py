@@ -52,6 +52,18 @@ MUTATIONS = [
     ("salient alpha_r of base 0", "const double ar = w->s_alpha_r[(size_t)k * M + i];\n        for (int64_t t",
      "const double ar = w->s_alpha_r[i];\n        for (int64_t t"),
     ("LUT alpha_r of base 0", "acc += w->alpha_r[(size_t)k * M + i] * s;", "acc += w->alpha_r[i] * s;"),
+    ("gather padding not zero", "            x_S[t] = 0.0;", "            x_S[t] = 1.0;"),
+    ("salient index bound off by one", "if ((int64_t)w->s_idx[t] >= w->N) return ORACLE_EINVAL;",
+     "if ((int64_t)w->s_idx[t] > w->N) return ORACLE_EINVAL;"),
+    ("more salient columns than columns accepted", "if (w->nS < 0 || w->nS > w->N) return ORACLE_EINVAL;",
+     "if (w->nS < 0) return ORACLE_EINVAL;"),
+    ("fp16 infinity read as NaN", "v = m ? NAN : INFINITY;", "v = NAN;"),
+    ("fp16 sign dropped", "return sign ? -v : v;", "return v;"),
+    ("dequantised row index", "dequant_row(w, i, Wout + (size_t)r * w->N);", "dequant_row(w, r, Wout + (size_t)r * w->N);"),
+    ("sampled row index", "            dequant_row(w, i, Wrow);", "            dequant_row(w, r, Wrow);"),
+    ("magnitude without x", "mag += fabs(Wrow[j] * xb[j]);", "mag += fabs(Wrow[j]);"),
+    ("salient groups rounded down", "const int64_t nSg = nS > 0 ? (nS + g - 1) / g * g : 0;",
+     "const int64_t nSg = nS > 0 ? nS / g * g : 0;"),
 ]
 
 
