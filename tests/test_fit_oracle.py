@@ -194,6 +194,13 @@ SOURCE_MUTATIONS = [
     ("salient residual not written back", "        R[:, S.astype(np.int64)] = RS\n", ""),
     ("salient bases fitted before the global ones", "    for k in range(K):\n        signs[k], alpha_r[k], alpha_c[k], R = fit_base(R, sweeps)\n",
      ""),
+    ("salient set shifted by one rank", "return np.sort(order[:nS]).astype(np.uint32)",
+     "return np.sort(order[1:nS + 1]).astype(np.uint32)"),
+    ("residual started from |W|", "    R = W.copy()\n", "    R = np.abs(W)\n"),
+    ("salient bases fitted to W", "RS = R[:, S.astype(np.int64)]", "RS = W[:, S.astype(np.int64)]"),
+    ("score as a sum", "return h * w", "return h + w"),
+    ("sweeps started from alpha_c = 2", "    ac = np.ones(N)\n", "    ac = np.full(N, 2.0)\n"),
+    ("residual update without the signs", "R_next = R - np.outer(ar, ac) * B", "R_next = R - np.outer(ar, ac) * np.abs(B)"),
 ]
 
 
