@@ -71,6 +71,9 @@ def test_hand_sized_case_by_loops():
     # by hand, row 0: group 0 = 1*1*1 + 2*(-1)*(-1) + 3*1*0.5 + 4*1*2 = 12.5, scaled by 2;
     # group 1 = 1*(-1)*4 + 1*(-1)*(-2) + 2*1*1 + 2*(-1)*0.25 = -0.5, scaled by 0.5
     assert want[0] == 24.75
+    # row 1: group 0 = 1*1*1 + 2*1*(-1) + 3*1*0.5 + 4*1*2 = 8.5, scaled by 1;
+    # group 1 = 1*(-1)*4 + 1*1*(-2) + 2*(-1)*1 + 2*1*0.25 = -7.5, scaled by 3
+    assert want[1] == -14.0
 
 
 def test_bad_grouping_is_rejected():
